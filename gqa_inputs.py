@@ -1,0 +1,120 @@
+"""Seeded synthetic inputs for the GQA prefill and decode workloads.
+
+This module is shared by the tests, the benchmark and the CPU oracle's callers.
+It only draws random numbers and describes shapes; it contains none of the
+attention arithmetic (no RoPE, no scores, no softmax), so that the oracle and
+the CUDA path share nothing but their inputs.
+
+Recipe (one seed per workload, ``seed = 1000 + workload index``):
+  * Q, K, V (and the decode caches) are drawn as float32 N(0, 1) from a
+    ``torch.Generator`` seeded with the workload's seed, in the order
+    q, k, v (prefill) or seqlens, q, kcache, vcache (decode), then rounded to
+    bfloat16 (round to nearest even).
+  * Decode cache lengths are uniform integers in [1, max_len].
+  * Shapes are the Qwen2 model shapes of the page "Qwen2 architecture
+    introduction" (aicoding.csdn.net), §4.4 Table 1: 0.5B 14/2 heads with head
+    size 64, 7B 28/4 heads with head size 128, 72B 64/8 heads with head size 128;
+    RoPE base 1e6 (same page, §5.2).
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass, field, replace
+
+import torch
+
+THETA = 1.0e6
+
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    kind: str            # "prefill" or "decode"
+    B: int
+    h_q: int
+    h_kv: int
+    d: int
+    L: int = 0           # prefill sequence length
+    max_len: int = 0     # decode: cache lengths are uniform in [1, max_len]
+    theta: float = THETA
+    seed: int = 0
+    desc: str = field(default="", compare=False)
+
+    @property
+    def g(self) -> int:
+        return self.h_q // self.h_kv
+
+    def with_(self, **kw) -> "Workload":
+        return replace(self, **kw)
+
+
+# The five workloads, in their canonical order (the index fixes the seed).
+WORKLOADS = [
+    Workload("qwen2-0.5b-prefill-L128", "prefill", B=1, L=128, h_q=14, h_kv=2, d=64,
+             desc="Qwen2-0.5B-shaped single-layer GQA prefill, B=1 L=128 h_q=14 h_kv=2 d=64"),
+    Workload("qwen2-7b-prefill-L4096", "prefill", B=1, L=4096, h_q=28, h_kv=4, d=128,
+             desc="Qwen2-7B-shaped GQA prefill, B=1 L=4096 h_q=28 h_kv=4 d=128"),
+    Workload("qwen2-72b-prefill-B4-L8192", "prefill", B=4, L=8192, h_q=64, h_kv=8, d=128,
+             desc="Qwen2-72B-shaped GQA prefill, B=4 L=8192 h_q=64 h_kv=8 d=128"),
+    Workload("qwen2-7b-decode-B64", "decode", B=64, max_len=32768, h_q=28, h_kv=4, d=128,
+             desc="Qwen2-7B-shaped GQA decode, B=64, cache lengths uniform in [1, 32768], h_q=28 h_kv=4 d=128"),
+    Workload("qwen2-7b-prefill-L32768", "prefill", B=1, L=32768, h_q=28, h_kv=4, d=128,
+             desc="Qwen2-7B-shaped long-context GQA prefill, B=1 L=32768 h_q=28 h_kv=4 d=128"),
+]
+WORKLOADS = [w.with_(seed=1000 + i) for i, w in enumerate(WORKLOADS)]
+BY_NAME = {w.name: w for w in WORKLOADS}
+
+
+def _gen(seed: int, device: str = "cpu") -> torch.Generator:
+    g = torch.Generator(device=device)
+    g.manual_seed(int(seed))
+    return g
+
+
+def _randn_bf16(shape, gen, device="cpu", chunk_rows=1 << 16):
+    """N(0,1) float32 rounded to bf16; drawn in leading-dim chunks to bound host memory."""
+    out = torch.empty(shape, dtype=torch.bfloat16, device=device)
+    n0 = shape[0]
+    for s in range(0, n0, chunk_rows):
+        e = min(n0, s + chunk_rows)
+        out[s:e] = torch.randn((e - s,) + tuple(shape[1:]), generator=gen,
+                               dtype=torch.float32, device=device).to(torch.bfloat16)
+    return out
+
+
+def prefill_inputs(w: Workload, device: str = "cpu"):
+    """q [B,L,h_q,d], k [B,L,h_kv,d], v [B,L,h_kv,d], all bf16, token-major."""
+    assert w.kind == "prefill"
+    gen = _gen(w.seed, device)
+    q = _randn_bf16((w.B * w.L, w.h_q, w.d), gen, device).view(w.B, w.L, w.h_q, w.d)
+    k = _randn_bf16((w.B * w.L, w.h_kv, w.d), gen, device).view(w.B, w.L, w.h_kv, w.d)
+    v = _randn_bf16((w.B * w.L, w.h_kv, w.d), gen, device).view(w.B, w.L, w.h_kv, w.d)
+    return q, k, v
+
+
+def decode_inputs(w: Workload, device: str = "cpu", seqlens=None):
+    """seqlens int32 [B]; q [B,h_q,d]; kcache, vcache packed [sum(seqlens), h_kv, d].
+
+    Sequence b's cache rows sit at packed rows off_b .. off_b + seqlens[b] - 1,
+    with off_b the sum of the lengths before it. ``seqlens`` may be given to
+    override the drawn lengths (edge-case tests); the draw still happens so the
+    random stream stays the same.
+    """
+    assert w.kind == "decode"
+    gen = _gen(w.seed, device)
+    drawn = torch.randint(1, w.max_len + 1, (w.B,), generator=gen, dtype=torch.int64,
+                          device=device).to(torch.int32)
+    if seqlens is not None:
+        drawn = torch.as_tensor(seqlens, dtype=torch.int32, device=device)
+        assert drawn.numel() == w.B
+    total = int(drawn.sum().item())
+    q = _randn_bf16((w.B, w.h_q, w.d), gen, device)
+    kc = _randn_bf16((max(total, 0), w.h_kv, w.d), gen, device)
+    vc = _randn_bf16((max(total, 0), w.h_kv, w.d), gen, device)
+    return drawn, q, kc, vc
+
+
+def small(kind: str, B: int, h_q: int, h_kv: int, d: int, L: int = 0, max_len: int = 0,
+          seed: int = 7, theta: float = THETA, name: str = "") -> Workload:
+    """A small ad-hoc workload for tests (ragged sizes, special head counts)."""
+    return Workload(name or f"{kind}-B{B}-L{L or max_len}-hq{h_q}-hkv{h_kv}-d{d}", kind,
+                    B=B, L=L, max_len=max_len, h_q=h_q, h_kv=h_kv, d=d, theta=theta, seed=seed)

@@ -1,0 +1,199 @@
+"""Plain fp64 CPU oracle for Qwen2-style grouped-query causal self-attention.
+
+TEST INFRASTRUCTURE ONLY.  Nothing in the product path may import, call or
+execute this module: only ``tests/``, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / reference leg of ``bench.py`` use it.  It shares no code
+with the CUDA library; the two meet only through the seeded inputs of
+``gqa_inputs``.
+
+What it computes is the textbook definition, written out step by step in
+float64 with NumPy, with no blocking or fusion beyond splitting the query rows
+into independent blocks (each block is still the full materialised product):
+
+  1. RoPE on Q and K (page "Qwen2架构解析：GQA与MoE技术在大模型中的创新应用",
+     intelliparadigm.com, §2.3; page "Qwen2 architecture introduction",
+     aicoding.csdn.net, §3.5.2 and §4.1.3 step 3): every Q and K row at
+     position m is rotated, pair by pair, by the angle m * theta^(-2i/d),
+     with d the head size and theta the RoPE base (1e6, same page §5.2).
+     Pairing: dimension i with i + d/2 ("rotate half"); the rotation is the
+     ordinary positive-angle plane rotation, i.e. the complex product
+     (x_i + j x_{i+d/2}) * exp(j * m * theta^(-2i/d)).
+  2. Head grouping (aicoding.csdn.net page, §4.1.2): with g = h_q / h_kv,
+     query head t (1-based) reads KV group floor((t-1)/g) + 1; 0-based this is
+     u = t // g.
+  3. Scores, mask, softmax, weighted sum (aicoding.csdn.net page, §4.1.3
+     step 4): S = Q' K'^T / sqrt(d), S_ij = -inf where j > i, A = row softmax,
+     head_t = A V_u.  The output keeps the concatenated-heads layout of §4.1.3
+     step 5: out[b, i, t, :] is row i of head_t.
+  4. Decode (aicoding.csdn.net page, §4.1.3 closing paragraph; page "从 Qwen 1
+     到 Qwen 2", nxmr.cn, §2.4): the cache holds only the h_kv groups of
+     un-rotated K and V; one new query per sequence, at position
+     p = seqlens[b], attends to all seqlens[b] cached rows (positions
+     0 .. p-1).  ``include_self=True`` selects the other reading, where the
+     cache already holds the new token and the query sits at p - 1.
+
+Every function is pinned by ``tests/test_oracle_pins.py`` against closed forms,
+invariants the pages state and a brute-force restatement.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+
+def as_f64(x) -> np.ndarray:
+    """Upcast a torch tensor (any float dtype, CPU) or array to a float64 ndarray."""
+    if hasattr(x, "detach"):
+        x = x.detach().to("cpu").float().numpy()
+    return np.asarray(x, dtype=np.float64)
+
+
+def head_group(t: int, g: int) -> int:
+    """0-based KV group of 0-based query head t (aicoding.csdn.net page, §4.1.2)."""
+    return t // g
+
+
+def inv_freq(d: int, theta: float) -> np.ndarray:
+    """theta^(-2i/d) for i = 0 .. d/2 - 1 (intelliparadigm.com page, §2.3, with d the head size)."""
+    i = np.arange(d // 2, dtype=np.float64)
+    return np.power(float(theta), -2.0 * i / d)
+
+
+def rope(x: np.ndarray, positions, theta: float) -> np.ndarray:
+    """Rotate rows of x [..., P, H, d] at positions [P] (step 1 of the module docstring)."""
+    x = np.asarray(x, dtype=np.float64)
+    d = x.shape[-1]
+    h = d // 2
+    ang = np.asarray(positions, dtype=np.float64)[:, None] * inv_freq(d, theta)[None, :]
+    c = np.cos(ang)[:, None, :]
+    s = np.sin(ang)[:, None, :]
+    x1 = x[..., :h]
+    x2 = x[..., h:]
+    return np.concatenate([x1 * c - x2 * s, x2 * c + x1 * s], axis=-1)
+
+
+def rope_interleaved(x: np.ndarray, positions, theta: float) -> np.ndarray:
+    """The other common pairing (2i with 2i+1); used only to test the permutation identity."""
+    x = np.asarray(x, dtype=np.float64)
+    d = x.shape[-1]
+    ang = np.asarray(positions, dtype=np.float64)[:, None] * inv_freq(d, theta)[None, :]
+    c = np.cos(ang)[:, None, :]
+    s = np.sin(ang)[:, None, :]
+    xe = x[..., 0::2]
+    xo = x[..., 1::2]
+    out = np.empty_like(x)
+    out[..., 0::2] = xe * c - xo * s
+    out[..., 1::2] = xo * c + xe * s
+    return out
+
+
+def softmax_rows(s: np.ndarray) -> np.ndarray:
+    """Row softmax with the row maximum subtracted; -inf entries get weight 0."""
+    m = np.max(s, axis=-1, keepdims=True)
+    e = np.exp(s - m)
+    return e / np.sum(e, axis=-1, keepdims=True)
+
+
+def causal_weights(qr_rows: np.ndarray, row_pos: np.ndarray, kr: np.ndarray) -> np.ndarray:
+    """A = softmax(Q'K'^T/sqrt(d) + M) for the query rows at positions row_pos against keys 0..n-1.
+
+    qr_rows [R, d] (rotated), kr [n, d] (rotated); M_ij = -inf where key j > query position.
+    """
+    d = qr_rows.shape[-1]
+    s = (qr_rows @ kr.T) / np.sqrt(d)
+    j = np.arange(kr.shape[0])[None, :]
+    s = np.where(j > np.asarray(row_pos)[:, None], -np.inf, s)
+    return softmax_rows(s)
+
+
+def prefill_ref(q, k, v, theta: float, row_block: int = 1024) -> np.ndarray:
+    """Full causal GQA prefill.  q [B,L,h_q,d], k/v [B,L,h_kv,d]; returns float64 [B,L,h_q,d]."""
+    q = as_f64(q)
+    k = as_f64(k)
+    v = as_f64(v)
+    B, L, h_q, d = q.shape
+    h_kv = k.shape[2]
+    assert h_q % h_kv == 0
+    g = h_q // h_kv
+    pos = np.arange(L)
+    qr = rope(q, pos, theta)
+    kr = rope(k, pos, theta)
+    out = np.empty((B, L, h_q, d), dtype=np.float64)
+    for b in range(B):
+        for t in range(h_q):
+            u = head_group(t, g)
+            for r0 in range(0, L, row_block):
+                r1 = min(L, r0 + row_block)
+                rows = np.arange(r0, r1)
+                a = causal_weights(qr[b, r0:r1, t, :], rows, kr[b, :r1, u, :])
+                out[b, r0:r1, t, :] = a @ v[b, :r1, u, :]
+    return out
+
+
+def prefill_rows_ref(q, k, v, theta: float, b: int, t: int, rows) -> np.ndarray:
+    """Selected output rows out[b, rows, t, :] of the causal prefill (for full-size spot checks).
+
+    Only the key rows 0 .. max(rows) are touched, so this works at any L.
+    """
+    rows = np.asarray(rows, dtype=np.int64)
+    h_q = q.shape[2]
+    h_kv = k.shape[2]
+    d = q.shape[3]
+    u = head_group(t, h_q // h_kv)
+    n = int(rows.max()) + 1
+    qr = rope(as_f64(q[b, rows, t, :])[:, None, :], rows, theta)[:, 0, :]
+    kr = rope(as_f64(k[b, :n, u, :])[:, None, :], np.arange(n), theta)[:, 0, :]
+    a = causal_weights(qr, rows, kr)
+    return a @ as_f64(v[b, :n, u, :])
+
+
+def decode_one_ref(q_b, krows, vrows, theta: float, include_self: bool = False) -> np.ndarray:
+    """One sequence: q_b [h_q,d], cache rows krows/vrows [s,h_kv,d] -> float64 [h_q,d]."""
+    q_b = as_f64(q_b)
+    krows = as_f64(krows)
+    vrows = as_f64(vrows)
+    h_q, d = q_b.shape
+    s, h_kv, _ = krows.shape
+    g = h_q // h_kv
+    p = s - 1 if include_self else s
+    qr = rope(q_b[None, :, :], [p], theta)[0]
+    kr = rope(krows, np.arange(s), theta)
+    out = np.empty((h_q, d), dtype=np.float64)
+    for t in range(h_q):
+        u = head_group(t, g)
+        a = causal_weights(qr[t][None, :], np.array([p]), kr[:, u, :])
+        out[t] = (a @ vrows[:, u, :])[0]
+    return out
+
+
+def packed_offsets(seqlens) -> np.ndarray:
+    """off_b = sum of seqlens before b; length B+1 (the packed-cache row index of each sequence)."""
+    s = np.asarray(seqlens, dtype=np.int64).reshape(-1)
+    return np.concatenate([[0], np.cumsum(s)])
+
+
+def decode_ref(q, kcache, vcache, seqlens, theta: float, include_self: bool = False,
+               batch_rows=None) -> np.ndarray:
+    """Decode step over the packed cache.  q [B,h_q,d]; caches [sum(seqlens),h_kv,d].
+
+    Returns float64 [B,h_q,d], or [len(batch_rows),h_q,d] for a subset of sequences.
+    """
+    seq = [int(x) for x in (seqlens.tolist() if hasattr(seqlens, "tolist") else seqlens)]
+    off = packed_offsets(seq)
+    bs = range(len(seq)) if batch_rows is None else list(batch_rows)
+    outs = []
+    for b in bs:
+        o0, o1 = int(off[b]), int(off[b + 1])
+        outs.append(decode_one_ref(q[b], kcache[o0:o1], vcache[o0:o1], theta, include_self))
+    return np.stack(outs, axis=0)
+
+
+def prefill_flops(B: int, L: int, h_q: int, d: int) -> float:
+    """Causal-effective FLOP count: 2 GEMMs x 2 flops x d over the L(L+1)/2 unmasked pairs per head."""
+    return 4.0 * B * h_q * d * L * (L + 1) / 2.0
+
+
+def decode_bytes(seqlens, h_q: int, h_kv: int, d: int, elem: int = 2) -> float:
+    """Algorithmic bytes of one decode step: K and V rows read once, plus q read and out written."""
+    total = float(np.sum(np.asarray(seqlens, dtype=np.int64)))
+    B = len(np.asarray(seqlens).reshape(-1))
+    return total * h_kv * d * elem * 2 + 2.0 * B * h_q * d * elem
