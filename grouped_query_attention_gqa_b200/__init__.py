@@ -1,0 +1,8 @@
+"""B200-native Qwen2-style grouped-query causal attention (GQA) with RoPE.
+
+The computation lives in libgqa.so (hand-written sm_100a CUDA behind the C ABI of
+include/gqa.h); this package is its thin Python binding.
+"""
+from ._lib import (  # noqa: F401
+    GQAError, DEVERR_SEQLEN, DEVERR_TIMEOUT, LIB_PATH, decode, last_error, load, prefill, release, strerror,
+)

@@ -1,0 +1,137 @@
+"""ctypes binding of libgqa (include/gqa.h).
+
+Argument marshalling only: shape/dtype/device checks, output allocation with torch,
+the current torch stream, and the C call.  Every step of the computation runs in the
+CUDA kernels of libgqa.so; there is no fallback path.  If the library is missing, the
+first call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libgqa.so")
+
+GQA_OK = 0
+DEVERR_SEQLEN = 1
+DEVERR_TIMEOUT = 2
+
+_lib = None
+
+
+class GQAError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        self.code = code
+        super().__init__(f"{what} failed with code {code}: {strerror(code)}")
+
+
+def load() -> ctypes.CDLL:
+    """Load libgqa.so (built by grouped_query_attention_gqa_b200.build); raise if absent."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                           f"`python -m grouped_query_attention_gqa_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+    lib.gqa_prefill.argtypes = [vp, vp, vp, vp, i, i, i, i, i, f]
+    lib.gqa_prefill.restype = i
+    lib.gqa_decode.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f]
+    lib.gqa_decode.restype = i
+    lib.gqa_set_stream.argtypes = [vp]
+    lib.gqa_set_stream.restype = i
+    lib.gqa_last_error.argtypes = []
+    lib.gqa_last_error.restype = i
+    lib.gqa_release.argtypes = []
+    lib.gqa_release.restype = None
+    lib.gqa_strerror.argtypes = [i]
+    lib.gqa_strerror.restype = ctypes.c_char_p
+    lib.gqa_abi_version.argtypes = []
+    lib.gqa_abi_version.restype = i
+    _lib = lib
+    return lib
+
+
+def strerror(code: int) -> str:
+    return load().gqa_strerror(int(code)).decode()
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _check(t, name, shape, dtype=torch.bfloat16):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+def _stream(device) -> None:
+    load().gqa_set_stream(ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream))
+
+
+def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, theta: float = 1.0e6,
+            out: torch.Tensor | None = None) -> torch.Tensor:
+    """Causal GQA prefill.  q [B,L,h_q,d], k/v [B,L,h_kv,d] bf16 CUDA -> out [B,L,h_q,d] bf16."""
+    if q.dim() != 4 or k.dim() != 4:
+        raise ValueError("q and k must be 4-D [B, L, heads, d]")
+    B, L, h_q, d = q.shape
+    h_kv = k.shape[2]
+    _check(q, "q", None)
+    _check(k, "k", (B, L, h_kv, d))
+    _check(v, "v", (B, L, h_kv, d))
+    if out is None:
+        out = torch.empty_like(q)
+    _check(out, "out", (B, L, h_q, d))
+    with torch.cuda.device(q.device):
+        _stream(q.device)
+        rc = load().gqa_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, L, h_q, h_kv, d, float(theta))
+    if rc != GQA_OK:
+        raise GQAError(rc, "gqa_prefill")
+    return out
+
+
+def decode(q: torch.Tensor, kcache: torch.Tensor, vcache: torch.Tensor, seqlens: torch.Tensor,
+           theta: float = 1.0e6, out: torch.Tensor | None = None) -> torch.Tensor:
+    """One decode step.  q [B,h_q,d]; caches packed [sum(seqlens),h_kv,d]; seqlens int32 [B] (device)."""
+    if q.dim() != 3 or kcache.dim() != 3:
+        raise ValueError("q must be [B, h_q, d] and kcache [rows, h_kv, d]")
+    B, h_q, d = q.shape
+    h_kv = kcache.shape[1]
+    _check(q, "q", None)
+    _check(kcache, "kcache", (kcache.shape[0], h_kv, d))
+    _check(vcache, "vcache", tuple(kcache.shape))
+    _check(seqlens, "seqlens", (B,), dtype=torch.int32)
+    if out is None:
+        out = torch.empty_like(q)
+    _check(out, "out", (B, h_q, d))
+    with torch.cuda.device(q.device):
+        _stream(q.device)
+        rc = load().gqa_decode(_ptr(q), _ptr(kcache), _ptr(vcache), _ptr(seqlens), _ptr(out),
+                               B, h_q, h_kv, d, float(theta))
+    if rc != GQA_OK:
+        raise GQAError(rc, "gqa_decode")
+    return out
+
+
+def last_error(device=None) -> int:
+    """Synchronise and return/clear the device error word (GQA_DEVERR_* bits)."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    with torch.cuda.device(dev):
+        _stream(dev)
+        return int(load().gqa_last_error())
+
+
+def release() -> None:
+    load().gqa_release()

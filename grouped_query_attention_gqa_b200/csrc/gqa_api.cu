@@ -1,0 +1,310 @@
+// libgqa: the C ABI declared in include/gqa.h.  Host-side validation, workspace
+// management, tensor-map encoding and kernel launches.  All kernels live in the
+// headers included below, so this is the library's single translation unit.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+
+#include "../../include/gqa.h"
+#include "decode_sm100.cuh"
+#include "prefill_sm100.cuh"
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+// The device error word (GQA_DEVERR_* bits), one per device context.
+__device__ int g_dev_err;
+
+struct DeviceState {
+    bool checked = false;
+    bool supported = false;
+    int num_sms = 0;
+    int* err = nullptr;           // device address of g_dev_err
+    void* ws = nullptr;           // prefill workspace
+    size_t ws_bytes = 0;
+    void* dws = nullptr;          // decode workspace
+    size_t dws_bytes = 0;
+};
+
+DeviceState g_dev[kMaxDevices];
+cudaStream_t g_stream = nullptr;
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+
+// Current device's state, after a one-time check that it is an sm_100 part.
+DeviceState* device_state(int* code) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        *code = GQA_ERR_DEVICE;
+        return nullptr;
+    }
+    DeviceState& st = g_dev[dev];
+    if (!st.checked) {
+        st.checked = true;
+        cudaDeviceProp prop;
+        if (cudaGetDeviceProperties(&prop, dev) == cudaSuccess && prop.major == 10 && prop.minor == 0) {
+            st.num_sms = prop.multiProcessorCount;
+            void* sym = nullptr;
+            if (cudaGetSymbolAddress(&sym, g_dev_err) == cudaSuccess) {
+                st.err = static_cast<int*>(sym);
+                st.supported = true;
+            }
+        }
+    }
+    if (!st.supported) {
+        *code = GQA_ERR_DEVICE;
+        return nullptr;
+    }
+    *code = GQA_OK;
+    return &st;
+}
+
+// Grow-only workspace.  A grow synchronises the stream first so that no queued kernel still
+// uses the old buffer.
+bool ensure(void*& ptr, size_t& have, size_t need) {
+    if (have >= need) return true;
+    if (ptr) {
+        cudaStreamSynchronize(g_stream);
+        cudaFree(ptr);
+        ptr = nullptr;
+        have = 0;
+    }
+    need = (need + 255) & ~size_t(255);
+    if (cudaMalloc(&ptr, need) != cudaSuccess) {
+        cudaGetLastError();
+        ptr = nullptr;
+        return false;
+    }
+    have = need;
+    return true;
+}
+
+bool get_encoder() {
+    if (g_encode) return true;
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || fn == nullptr)
+        return false;
+    g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+    return true;
+}
+
+// bf16 tensor map: innermost dimension d, box {64, ..., 128 rows, ...}, 128-byte swizzle.
+bool encode_bf16(CUtensorMap* map, const void* base, int rank, const cuuint64_t* dims, const cuuint64_t* strides,
+                 const cuuint32_t* box) {
+    cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+    const CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims, strides,
+                                box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_common(int h_q, int h_kv, int d, float theta) {
+    if (h_q <= 0 || h_kv <= 0 || h_q % h_kv != 0) return GQA_ERR_DIMS;
+    if (d != 64 && d != 128) return GQA_ERR_HEAD_DIM;
+    if (!(theta > 0.0f) || !std::isfinite(theta)) return GQA_ERR_THETA;
+    return GQA_OK;
+}
+
+template <int D>
+int launch_prefill(DeviceState* st, const void* q, const void* k, const void* v, void* out, int B, int L, int h_q,
+                   int h_kv, float theta) {
+    using namespace gqa::prefill;
+    const size_t kr_bytes = static_cast<size_t>(B) * h_kv * L * D * 2;
+    const size_t cs_off = (kr_bytes + 255) & ~size_t(255);
+    const size_t need = cs_off + static_cast<size_t>(L) * (D / 2) * sizeof(float2);
+    if (!ensure(st->ws, st->ws_bytes, need)) return GQA_ERR_ALLOC;
+    auto* kr = static_cast<__nv_bfloat16*>(st->ws);
+    auto* cs = reinterpret_cast<float2*>(static_cast<uint8_t*>(st->ws) + cs_off);
+
+    if (!get_encoder()) return GQA_ERR_LAUNCH;
+    CUtensorMap tm_k, tm_v;
+    {   // K' [B*h_kv, L, D]
+        const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(L),
+                                    static_cast<cuuint64_t>(B) * h_kv};
+        const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(L) * D * 2};
+        const cuuint32_t box[3] = {64, BN, 1};
+        if (!encode_bf16(&tm_k, kr, 3, dims, strides, box)) return GQA_ERR_LAUNCH;
+    }
+    {   // V [B, L, h_kv, D]
+        const cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(h_kv),
+                                    static_cast<cuuint64_t>(L), static_cast<cuuint64_t>(B)};
+        const cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(h_kv) * D * 2,
+                                       static_cast<cuuint64_t>(L) * h_kv * D * 2};
+        const cuuint32_t box[4] = {64, 1, BN, 1};
+        if (!encode_bf16(&tm_v, v, 4, dims, strides, box)) return GQA_ERR_LAUNCH;
+    }
+
+    const int prep_blocks = (L + PREP_POS - 1) / PREP_POS;
+    prep_kernel<D><<<prep_blocks, PREP_THREADS, 0, g_stream>>>(static_cast<const __nv_bfloat16*>(k), kr, cs, B, L,
+                                                               h_kv, static_cast<double>(theta));
+    if (cudaGetLastError() != cudaSuccess) return GQA_ERR_LAUNCH;
+
+    Params p;
+    p.q = static_cast<const __nv_bfloat16*>(q);
+    p.out = static_cast<__nv_bfloat16*>(out);
+    p.cs = cs;
+    p.B = B;
+    p.L = L;
+    p.h_q = h_q;
+    p.h_kv = h_kv;
+    p.g = h_q / h_kv;
+    p.n_qtiles = (L + BM - 1) / BM;
+    p.tiles_per_group = p.n_qtiles * p.g;
+    p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
+    p.err = st->err;
+    const int pairs = (p.tiles_per_group + 1) / 2;
+    const long long grid = static_cast<long long>(pairs) * B * h_kv;
+    if (grid > 0x7fffffffLL) return GQA_ERR_DIMS;
+    if (cudaFuncSetAttribute(attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, Layout<D>::DYN) !=
+        cudaSuccess)
+        return GQA_ERR_LAUNCH;
+    // The in-kernel register split (setmaxnreg) is only valid for this exact launch budget.
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, attn_kernel<D>) != cudaSuccess || fa.numRegs != LAUNCH_REGS)
+        return GQA_ERR_LAUNCH;
+    attn_kernel<D><<<static_cast<unsigned>(grid), NUM_THREADS, Layout<D>::DYN, g_stream>>>(tm_k, tm_v, p);
+    if (cudaGetLastError() != cudaSuccess) return GQA_ERR_LAUNCH;
+    return GQA_OK;
+}
+
+template <int D>
+int launch_decode(DeviceState* st, const void* q, const void* kc, const void* vc, const int* seqlens, void* out,
+                  int B, int h_q, int h_kv, float theta) {
+    using namespace gqa::decode;
+    using C = Cfg<D>;
+    const int g = h_q / h_kv;
+    const int n_hb = (g + HB - 1) / HB;
+    const int groups = h_kv * n_hb;
+    // About two CTAs of WARPS workers per SM in total, split evenly over the (group, head block) pairs.
+    const int G = (2 * st->num_sms + groups - 1) / groups;
+    const int P = G * WARPS;
+    const size_t off_bytes = (static_cast<size_t>(B + 1) * sizeof(int64_t) + 255) & ~size_t(255);
+    const size_t part_bytes = static_cast<size_t>(P + B) * groups * C::PART * sizeof(float);
+    if (!ensure(st->dws, st->dws_bytes, off_bytes + part_bytes)) return GQA_ERR_ALLOC;
+
+    Params p;
+    p.q = static_cast<const __nv_bfloat16*>(q);
+    p.kc = static_cast<const __nv_bfloat16*>(kc);
+    p.vc = static_cast<const __nv_bfloat16*>(vc);
+    p.out = static_cast<__nv_bfloat16*>(out);
+    p.off = static_cast<int64_t*>(st->dws);
+    p.part = reinterpret_cast<float*>(static_cast<uint8_t*>(st->dws) + off_bytes);
+    p.B = B;
+    p.h_q = h_q;
+    p.h_kv = h_kv;
+    p.g = g;
+    p.n_hb = n_hb;
+    p.P = P;
+    p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
+    p.theta = static_cast<double>(theta);
+    p.err = st->err;
+
+    plan_kernel<<<1, PLAN_THREADS, 0, g_stream>>>(seqlens, static_cast<int64_t*>(st->dws), B, st->err);
+    if (cudaGetLastError() != cudaSuccess) return GQA_ERR_LAUNCH;
+    if (cudaFuncSetAttribute(split_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
+        return GQA_ERR_LAUNCH;
+    split_kernel<D><<<G * groups, WARPS * 32, C::SMEM, g_stream>>>(p);
+    if (cudaGetLastError() != cudaSuccess) return GQA_ERR_LAUNCH;
+    const long long cgrid = static_cast<long long>(B) * groups;
+    if (cgrid > 0x7fffffffLL) return GQA_ERR_DIMS;
+    combine_kernel<D><<<static_cast<unsigned>(cgrid), COMBINE_THREADS, 0, g_stream>>>(p);
+    if (cudaGetLastError() != cudaSuccess) return GQA_ERR_LAUNCH;
+    return GQA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int gqa_abi_version(void) { return 1; }
+
+const char* gqa_strerror(int code) {
+    switch (code) {
+        case GQA_OK: return "success";
+        case GQA_ERR_NULL: return "a required pointer is NULL";
+        case GQA_ERR_DIMS: return "invalid sizes (negative, h_q not a multiple of h_kv, or too large)";
+        case GQA_ERR_HEAD_DIM: return "unsupported head dimension (must be 64 or 128)";
+        case GQA_ERR_THETA: return "RoPE base theta must be positive and finite";
+        case GQA_ERR_LAUNCH: return "CUDA launch or tensor-map encoding failed";
+        case GQA_ERR_ALLOC: return "workspace allocation failed";
+        case GQA_ERR_ALIGN: return "a tensor pointer is not 16-byte aligned";
+        case GQA_ERR_DEVICE: return "the current CUDA device is not an sm_100 GPU";
+        default: return "unknown error code";
+    }
+}
+
+int gqa_set_stream(void* cuda_stream) {
+    g_stream = static_cast<cudaStream_t>(cuda_stream);
+    return GQA_OK;
+}
+
+int gqa_prefill(const void* q, const void* k, const void* v, void* out, int B, int L, int h_q, int h_kv, int d,
+                float theta) {
+    if (B < 0 || L < 0) return GQA_ERR_DIMS;
+    int rc = check_common(h_q, h_kv, d, theta);
+    if (rc != GQA_OK) return rc;
+    if (B == 0 || L == 0) return GQA_OK;
+    if (!q || !k || !v || !out) return GQA_ERR_NULL;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return GQA_ERR_ALIGN;
+    // TMA coordinates are 32-bit and the kernel indexes rows with 32-bit positions.
+    if (static_cast<long long>(B) * h_kv > 0x7fffffffLL || L > (1 << 30)) return GQA_ERR_DIMS;
+    DeviceState* st = device_state(&rc);
+    if (!st) return rc;
+    return d == 64 ? launch_prefill<64>(st, q, k, v, out, B, L, h_q, h_kv, theta)
+                   : launch_prefill<128>(st, q, k, v, out, B, L, h_q, h_kv, theta);
+}
+
+int gqa_decode(const void* q, const void* kcache, const void* vcache, const int* seqlens, void* out, int B, int h_q,
+               int h_kv, int d, float theta) {
+    if (B < 0) return GQA_ERR_DIMS;
+    int rc = check_common(h_q, h_kv, d, theta);
+    if (rc != GQA_OK) return rc;
+    if (B == 0) return GQA_OK;
+    if (!q || !kcache || !vcache || !seqlens || !out) return GQA_ERR_NULL;
+    if (!aligned16(q) || !aligned16(kcache) || !aligned16(vcache) || !aligned16(out)) return GQA_ERR_ALIGN;
+    DeviceState* st = device_state(&rc);
+    if (!st) return rc;
+    return d == 64 ? launch_decode<64>(st, q, kcache, vcache, seqlens, out, B, h_q, h_kv, theta)
+                   : launch_decode<128>(st, q, kcache, vcache, seqlens, out, B, h_q, h_kv, theta);
+}
+
+int gqa_last_error(void) {
+    int rc = GQA_OK;
+    DeviceState* st = device_state(&rc);
+    if (!st) return rc;
+    if (cudaStreamSynchronize(g_stream) != cudaSuccess) return GQA_ERR_LAUNCH;
+    int h = 0;
+    if (cudaMemcpyFromSymbol(&h, g_dev_err, sizeof(int)) != cudaSuccess) return GQA_ERR_LAUNCH;
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_dev_err, &zero, sizeof(int)) != cudaSuccess) return GQA_ERR_LAUNCH;
+    return h;
+}
+
+void gqa_release(void) {
+    int cur = 0;
+    if (cudaGetDevice(&cur) != cudaSuccess) return;
+    for (int dev = 0; dev < kMaxDevices; ++dev) {
+        DeviceState& st = g_dev[dev];
+        if (!st.ws && !st.dws) continue;
+        cudaSetDevice(dev);
+        cudaDeviceSynchronize();
+        if (st.ws) cudaFree(st.ws);
+        if (st.dws) cudaFree(st.dws);
+        st.ws = st.dws = nullptr;
+        st.ws_bytes = st.dws_bytes = 0;
+    }
+    cudaSetDevice(cur);
+}
+
+}  // extern "C"

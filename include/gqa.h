@@ -1,0 +1,108 @@
+/*
+ * gqa.h -- C ABI of libgqa: Qwen2-style grouped-query causal self-attention with RoPE
+ * on one NVIDIA B200 (sm_100a).
+ *
+ * The operation (page "Qwen2 architecture introduction", aicoding.csdn.net, §4.1.2-§4.1.3;
+ * page "Qwen2架构解析：GQA与MoE技术在大模型中的创新应用", intelliparadigm.com, §2.3 and §3.1):
+ *   g = h_q / h_kv query heads share each key/value head; query head t (0-based) reads
+ *   KV group u = t / g.  Q and K rows at position m are rotated (RoPE) pair by pair,
+ *   dimension i with i + d/2, by the angle m * theta^(-2i/d).  Per head,
+ *   S = Q' K'^T / sqrt(d), S_ij = -inf for j > i (causal), A = softmax(S), head_t = A V_u.
+ *
+ * Conventions for every entry point below
+ *   - All tensor pointers are DEVICE pointers owned by the caller, bf16 (bfloat16, stored
+ *     as 16-bit words), dense row-major with exactly the shapes given, 16-byte aligned.
+ *   - Work is enqueued on the stream set by gqa_set_stream() (default: the legacy stream 0)
+ *     and runs asynchronously; no call below synchronises the host except gqa_last_error()
+ *     and the first call on a device (one-time device query).
+ *   - Return value: 0 on success, or one of the negative GQA_ERR_* codes.  A failing call
+ *     launches nothing and leaves `out` untouched.  Library code never traps or aborts.
+ *   - Not thread-safe: the stream and the workspace are process-global state.
+ */
+#ifndef GQA_H_
+#define GQA_H_
+
+#if defined(__GNUC__)
+#define GQA_API __attribute__((visibility("default")))
+#else
+#define GQA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define GQA_OK 0
+#define GQA_ERR_NULL (-1)      /* a required pointer is NULL                                  */
+#define GQA_ERR_DIMS (-2)      /* B, L < 0; h_q, h_kv <= 0; h_q % h_kv != 0; or sizes too large */
+#define GQA_ERR_HEAD_DIM (-3)  /* d is not 64 or 128                                          */
+#define GQA_ERR_THETA (-4)     /* theta <= 0 or not finite                                    */
+#define GQA_ERR_LAUNCH (-5)    /* a CUDA launch or tensor-map encode failed                   */
+#define GQA_ERR_ALLOC (-6)     /* the internal workspace could not be allocated               */
+#define GQA_ERR_ALIGN (-7)     /* a tensor pointer is not 16-byte aligned                     */
+#define GQA_ERR_DEVICE (-8)    /* the current device is not an sm_100 (B200-class) GPU        */
+
+/* Bits of the device error word returned by gqa_last_error(). */
+#define GQA_DEVERR_SEQLEN 1    /* a decode length was <= 0; that sequence's output was zeroed */
+#define GQA_DEVERR_TIMEOUT 2   /* a kernel pipeline wait ran past its limit and gave up;     */
+                               /* outputs of that call are undefined                          */
+
+/*
+ * Causal GQA prefill over whole sequences (page "Qwen2 architecture introduction",
+ * §4.1.3 steps 3-5).
+ *   q   [B, L, h_q,  d]   token-major: the per-head split of the Q projection output
+ *   k   [B, L, h_kv, d]   un-rotated keys
+ *   v   [B, L, h_kv, d]
+ *   out [B, L, h_q,  d]   head_t rows, i.e. the concatenation [head_1 | ... | head_hq]
+ * Positions are 0 .. L-1 in every batch row.  d in {64, 128}; h_q % h_kv == 0; any L >= 1
+ * (a ragged last tile is handled).  B == 0 or L == 0 is a no-op that returns GQA_OK.
+ * Uses an internal device workspace (rotated K and a cos/sin table, about
+ * B*h_kv*L*d*2 + L*d*4 bytes), grown on demand and kept until gqa_release().
+ * theta is the RoPE base (Qwen2: 1e6).
+ */
+GQA_API int gqa_prefill(const void* q, const void* k, const void* v, void* out,
+                int B, int L, int h_q, int h_kv, int d, float theta);
+
+/*
+ * One decode step: one new query token per sequence against a packed KV cache
+ * (page "Qwen2 architecture introduction", §4.1.3 closing paragraph: only the h_kv groups
+ * are cached; page "从 Qwen 1 到 Qwen 2", nxmr.cn, §2.4).
+ *   q       [B, h_q, d]
+ *   kcache  [sum(seqlens), h_kv, d]   un-rotated keys, sequences concatenated in b order:
+ *   vcache  [sum(seqlens), h_kv, d]   row j of sequence b is packed row off_b + j,
+ *                                     off_b = seqlens[0] + ... + seqlens[b-1]
+ *   seqlens [B] int32, DEVICE memory; each >= 1
+ *   out     [B, h_q, d]
+ * The query of sequence b sits at position seqlens[b] and attends to all seqlens[b] cached
+ * rows (positions 0 .. seqlens[b]-1).  A length <= 0 is not an API error (lengths live on
+ * the device): that sequence's output is zeroed and GQA_DEVERR_SEQLEN is raised in the device
+ * error word.  B == 0 is a no-op.  Uses an internal workspace (packed offsets and split
+ * partials, a few MB), grown on demand and kept until gqa_release().
+ */
+GQA_API int gqa_decode(const void* q, const void* kcache, const void* vcache, const int* seqlens,
+               void* out, int B, int h_q, int h_kv, int d, float theta);
+
+/* Stream for subsequent calls (a cudaStream_t passed as void*; NULL = legacy stream). */
+GQA_API int gqa_set_stream(void* cuda_stream);
+
+/*
+ * Synchronises the current stream, then returns and clears the device error word of the
+ * current device (a combination of GQA_DEVERR_* bits; 0 if clean), or GQA_ERR_LAUNCH if
+ * the stream reports a CUDA error.
+ */
+GQA_API int gqa_last_error(void);
+
+/* Frees the internal workspaces of every device this process used (synchronises each). */
+GQA_API void gqa_release(void);
+
+/* Static, human-readable text for a GQA_ERR_* code. */
+GQA_API const char* gqa_strerror(int code);
+
+/* ABI version of this header (incremented on incompatible changes). */
+GQA_API int gqa_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GQA_H_ */

@@ -1,0 +1,92 @@
+"""The C-ABI library loads, exports every entry point include/gqa.h declares, and validates
+its arguments on the host (no GPU needed: every call here fails before any CUDA work)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import grouped_query_attention_gqa_b200 as G
+from grouped_query_attention_gqa_b200 import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "gqa.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return G.load()
+
+
+def declared():
+    txt = open(HEADER).read()
+    return re.findall(r"GQA_API\s+[\w\s\*]+?\b(gqa_\w+)\s*\(", txt)
+
+
+def codes():
+    txt = open(HEADER).read()
+    return {m[0]: int(m[1]) for m in re.findall(r"#define (GQA_\w+) \(?(-?\d+)\)?", txt)}
+
+
+def test_header_declares_the_entry_points():
+    names = set(declared())
+    for n in ["gqa_prefill", "gqa_decode", "gqa_set_stream", "gqa_last_error", "gqa_release",
+              "gqa_strerror", "gqa_abi_version"]:
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared():
+        assert hasattr(lib, name), f"{name} declared in gqa.h but not exported"
+
+
+def test_version_and_strerror(lib):
+    assert lib.gqa_abi_version() == 1
+    c = codes()
+    for k, v in c.items():
+        if k.startswith("GQA_ERR_"):
+            assert G.strerror(v) != "unknown error code"
+    assert G.strerror(12345) == "unknown error code"
+
+
+F = ctypes.c_float(1.0e6)
+P16 = ctypes.c_void_p(256)
+
+
+@pytest.mark.parametrize("args,code", [
+    ((P16, P16, P16, P16, -1, 16, 28, 4, 128, F), "GQA_ERR_DIMS"),
+    ((P16, P16, P16, P16, 1, -3, 28, 4, 128, F), "GQA_ERR_DIMS"),
+    ((P16, P16, P16, P16, 1, 16, 28, 5, 128, F), "GQA_ERR_DIMS"),
+    ((P16, P16, P16, P16, 1, 16, 0, 4, 128, F), "GQA_ERR_DIMS"),
+    ((P16, P16, P16, P16, 1, 16, 28, 0, 128, F), "GQA_ERR_DIMS"),
+    ((P16, P16, P16, P16, 1, 16, 28, 4, 96, F), "GQA_ERR_HEAD_DIM"),
+    ((P16, P16, P16, P16, 1, 16, 28, 4, 128, ctypes.c_float(0.0)), "GQA_ERR_THETA"),
+    ((P16, P16, P16, P16, 1, 16, 28, 4, 128, ctypes.c_float(float("inf"))), "GQA_ERR_THETA"),
+    ((P16, P16, P16, P16, 1, 16, 28, 4, 128, ctypes.c_float(float("nan"))), "GQA_ERR_THETA"),
+    ((None, P16, P16, P16, 1, 16, 28, 4, 128, F), "GQA_ERR_NULL"),
+    ((P16, P16, P16, None, 1, 16, 28, 4, 128, F), "GQA_ERR_NULL"),
+    ((P16, P16, ctypes.c_void_p(264), P16, 1, 16, 28, 4, 128, F), "GQA_ERR_ALIGN"),
+    ((None, None, None, None, 0, 16, 28, 4, 128, F), "GQA_OK"),      # empty batch: no-op
+    ((None, None, None, None, 2, 0, 28, 4, 128, F), "GQA_OK"),       # empty sequence: no-op
+])
+def test_prefill_validation(lib, args, code):
+    assert lib.gqa_prefill(*args) == codes()[code]
+
+
+@pytest.mark.parametrize("args,code", [
+    ((P16, P16, P16, P16, P16, -1, 28, 4, 128, F), "GQA_ERR_DIMS"),
+    ((P16, P16, P16, P16, P16, 4, 28, 3, 128, F), "GQA_ERR_DIMS"),
+    ((P16, P16, P16, P16, P16, 4, 28, 4, 32, F), "GQA_ERR_HEAD_DIM"),
+    ((P16, P16, P16, P16, P16, 4, 28, 4, 64, ctypes.c_float(-1.0)), "GQA_ERR_THETA"),
+    ((P16, P16, P16, None, P16, 4, 28, 4, 128, F), "GQA_ERR_NULL"),
+    ((P16, None, P16, P16, P16, 4, 28, 4, 128, F), "GQA_ERR_NULL"),
+    ((ctypes.c_void_p(260), P16, P16, P16, P16, 4, 28, 4, 128, F), "GQA_ERR_ALIGN"),
+    ((None, None, None, None, None, 0, 28, 4, 128, F), "GQA_OK"),
+])
+def test_decode_validation(lib, args, code):
+    assert lib.gqa_decode(*args) == codes()[code]
+
+
+def test_set_stream_accepts_null(lib):
+    assert lib.gqa_set_stream(None) == 0

@@ -1,0 +1,106 @@
+"""GPU prefill (libgqa through its C ABI) against the fp64 oracle."""
+import numpy as np
+import pytest
+import torch
+
+import gqa_inputs as gi
+from oracle import gqa_ref as R
+from tests.parity_util import assert_close
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def G():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from grouped_query_attention_gqa_b200 import build
+    build.build()
+    import grouped_query_attention_gqa_b200 as G
+    return G
+
+
+def run(G, q, k, v, theta):
+    dev = torch.device("cuda")
+    out = G.prefill(q.to(dev), k.to(dev), v.to(dev), theta=theta)
+    assert G.last_error() == 0
+    return out.float().cpu().numpy()
+
+
+SMALL = [
+    # (B, L, h_q, h_kv, d)  -- several tiles, ragged tails, GQA / MHA / MQA, both head sizes
+    (1, 128, 14, 2, 64),
+    (1, 1, 14, 2, 64),
+    (2, 5, 4, 2, 128),
+    (1, 127, 7, 1, 128),
+    (1, 129, 8, 8, 128),
+    (2, 300, 14, 2, 64),
+    (1, 513, 28, 4, 128),
+    (3, 200, 16, 4, 128),
+    (1, 1000, 4, 1, 64),
+]
+
+
+@pytest.mark.parametrize("B,L,h_q,h_kv,d", SMALL)
+def test_prefill_small_full_output(G, B, L, h_q, h_kv, d):
+    w = gi.small("prefill", B=B, L=L, h_q=h_q, h_kv=h_kv, d=d, seed=B * 1000 + L + h_q)
+    q, k, v = gi.prefill_inputs(w)
+    got = run(G, q, k, v, w.theta)
+    ref = R.prefill_ref(q, k, v, w.theta)
+    assert_close(got, ref, f"prefill B={B} L={L} h_q={h_q} h_kv={h_kv} d={d}")
+
+
+def test_prefill_first_row_is_v0_exactly(G):
+    w = gi.small("prefill", B=2, L=300, h_q=28, h_kv=4, d=128, seed=5)
+    q, k, v = gi.prefill_inputs(w)
+    got = run(G, q, k, v, w.theta)
+    vv = v.float().numpy()
+    for t in range(28):
+        assert np.array_equal(got[:, 0, t], vv[:, 0, t // 7])
+
+
+def test_prefill_gqa_equals_mha_on_expanded_kv(G):
+    """The kernel's head->group map against the repeat_interleave expansion, both on the GPU."""
+    w = gi.small("prefill", B=1, L=260, h_q=28, h_kv=4, d=128, seed=9)
+    q, k, v = gi.prefill_inputs(w)
+    a = run(G, q, k, v, w.theta)
+    b = run(G, q, k.repeat_interleave(7, dim=2).contiguous(), v.repeat_interleave(7, dim=2).contiguous(),
+            w.theta)
+    assert np.array_equal(a, b)
+
+
+def test_prefill_theta_1e4_and_repeat_calls(G):
+    w = gi.small("prefill", B=1, L=384, h_q=8, h_kv=2, d=128, seed=11, theta=1.0e4)
+    q, k, v = gi.prefill_inputs(w)
+    ref = R.prefill_ref(q, k, v, w.theta)
+    for _ in range(2):
+        assert_close(run(G, q, k, v, w.theta), ref, "theta=1e4")
+
+
+def sample_rows(L, rng, n=24):
+    fixed = {0, 1, 127, 128, 129, 255, 256, L // 2, L - 2, L - 1}
+    rows = {r for r in fixed if 0 <= r < L} | set(rng.integers(0, L, n).tolist())
+    return np.array(sorted(rows))
+
+
+@pytest.mark.parametrize("name", ["qwen2-0.5b-prefill-L128", "qwen2-7b-prefill-L4096",
+                                  "qwen2-72b-prefill-B4-L8192", "qwen2-7b-prefill-L32768"])
+def test_prefill_full_size_sampled_rows(G, name):
+    """Full workload sizes, same launch as the benchmark; the oracle checks sampled rows."""
+    w = gi.BY_NAME[name]
+    q, k, v = gi.prefill_inputs(w)
+    dev = torch.device("cuda")
+    out = G.prefill(q.to(dev), k.to(dev), v.to(dev), theta=w.theta)
+    assert G.last_error() == 0
+    rng = np.random.default_rng(w.seed)
+    heads = sorted({0, w.h_q - 1, w.g, *rng.integers(0, w.h_q, 3).tolist()})
+    vv = v[:, 0].float().numpy()
+    row0 = out[:, 0].float().cpu().numpy()
+    for t in range(w.h_q):   # row 0 of every head is v_0 of its group, exactly
+        assert np.array_equal(row0[:, t], vv[:, t // w.g])
+    for b in sorted({0, w.B - 1}):
+        for t in heads:
+            rows = sample_rows(w.L, rng)
+            got = out[b, torch.as_tensor(rows, device=dev), t].float().cpu().numpy()
+            ref = R.prefill_rows_ref(q, k, v, w.theta, b, t, rows)
+            assert_close(got, ref, f"{name} b={b} t={t}")
