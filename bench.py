@@ -1,0 +1,443 @@
+#!/usr/bin/env python
+"""Benchmark of the GQA hot path on B200: prefill TFLOP/s and decode KV-cache GB/s.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+    torchrun --nproc-per-node N bench.py --gpus N ...      (one process per GPU)
+
+One step is one pass of the whole hot path: a causal prefill over the Qwen2-7B-shaped workload
+(B=1, L=4096, 28/4 heads, d=128) followed by one decode step over the Qwen2-7B-shaped decode
+workload (B=64 sequences, cache lengths uniform in [1, 32768]).  The headline `value` is the
+prefill's causal-effective TFLOP/s (4*B*h_q*d*L(L+1)/2 per step, summed over ranks, divided by
+the slowest rank's device time); the decode step is reported beside it in GB/s of KV cache.
+Inputs are synthetic (seeded N(0,1) bf16, drawn on the device) and resident in HBM when the
+timed region starts; the L2 is flushed (a 256 MiB write) before every prefill, and the decode
+cache (~2.1 GB) is far larger than L2.  Each rank of an N-GPU run processes its own copy of
+the workload (independent batches, no collective on the data path: weak scaling).
+
+`--impl reference` times the plain fp64 CPU oracle (the only reference that exists for this
+method) on a bounded sample of the same prefill workload, on the host cores of rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import glob
+import hashlib
+import json
+import os
+import re
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+import gqa_inputs as gi  # noqa: E402
+
+METRIC = "GQA prefill TFLOP/s & decode KV GB/s, as % of B200 tensor/HBM peak"
+PREFILL_WORKLOAD = "qwen2-7b-prefill-L4096"
+DECODE_WORKLOAD = "qwen2-7b-decode-B64"
+FLUSH_BYTES = 256 << 20
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ------------------------------------------------------------------------------------------ helpers
+def prefill_flops(w) -> float:
+    return 4.0 * w.B * w.h_q * w.d * w.L * (w.L + 1) / 2.0
+
+
+def decode_kv_bytes(total_rows: int, w) -> float:
+    return float(total_rows) * w.h_kv * w.d * 2 * 2
+
+
+def decode_bytes(total_rows: int, w) -> float:
+    return decode_kv_bytes(total_rows, w) + 2.0 * w.B * w.h_q * w.d * 2
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def source_sha() -> str:
+    """Hash of the library sources; a profile's DRAM traffic is used only while it matches."""
+    h = hashlib.sha256()
+    files = sorted(glob.glob(os.path.join(ROOT, "grouped_query_attention_gqa_b200", "csrc", "*.cu*")))
+    files.append(os.path.join(ROOT, "include", "gqa.h"))
+    for fn in files:
+        with open(fn, "rb") as f:
+            h.update(os.path.basename(fn).encode() + b"\0" + f.read())
+    return h.hexdigest()[:16]
+
+
+def profile_traffic(key: str):
+    """DRAM bytes per launch of kernel `key` from the committed ncu summaries, if still current."""
+    sha = source_sha()
+    for fn in sorted(glob.glob(os.path.join(ROOT, "profiles", "*.md"))):
+        txt = open(fn, encoding="utf-8").read()
+        m_sha = re.search(r"source_sha256_16:\s*([0-9a-f]{16})", txt)
+        m_tr = re.search(r"traffic_bytes_per_launch\[" + re.escape(key) + r"\]:\s*([0-9.eE+]+)", txt)
+        if m_sha and m_tr and m_sha.group(1) == sha:
+            return float(m_tr.group(1))
+    return None
+
+
+class ClockSampler:
+    """Polls NVML for SM clock and clock-event reasons on a background thread."""
+
+    NAMES = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+             0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+             0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+    def __init__(self, device_index: int, period_s: float = 0.002):
+        self.samples, self.reasons, self.ok = [], 0, False
+        self.period = period_s
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            props = torch.cuda.get_device_properties(device_index)
+            bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByPciBusId(bus.encode())
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # NVML missing: report that instead of clocks
+            self.err = repr(e)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                self.reasons |= int(self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok:
+            return {"error": getattr(self, "err", "nvml unavailable")}
+        rs = [n for bit, n in self.NAMES.items() if self.reasons & bit and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "samples": len(self.samples), "reasons": rs}
+
+
+def clean(x):
+    """NaN/inf (a leg that did not run) -> None, so the line stays strict JSON."""
+    if isinstance(x, dict):
+        return {k: clean(v) for k, v in x.items()}
+    if isinstance(x, (list, tuple)):
+        return [clean(v) for v in x]
+    if isinstance(x, float) and (x != x or x in (float("inf"), float("-inf"))):
+        return None
+    return x
+
+
+# ------------------------------------------------------------------------------------------ ranks
+def dist_env():
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("LOCAL_RANK", 0)), int(os.environ.get("WORLD_SIZE", 1))
+
+
+def dist_init(world: int, backend: str = "nccl"):
+    if world > 1 and not torch.distributed.is_initialized():
+        torch.distributed.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+
+
+def reduce_max(x: float, device) -> float:
+    """Max of a scalar over all ranks (identity when not distributed)."""
+    if not (torch.distributed.is_available() and torch.distributed.is_initialized()):
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier():
+    if torch.distributed.is_available() and torch.distributed.is_initialized():
+        torch.distributed.barrier()
+
+
+# ------------------------------------------------------------------------------------------ CPU oracle
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def oracle_prefill_sample(w, budget_s: float, max_steps: int | None = None):
+    """Time the fp64 oracle on one-head slices of the prefill workload (heads in turn)."""
+    from oracle import gqa_ref as R
+    q, k, v = gi.prefill_inputs(w)
+    per_head = prefill_flops(w.with_(B=1, h_q=1, h_kv=1))
+    times, t0 = [], time.perf_counter()
+    t = 0
+    while True:
+        u = t // w.g
+        a = time.perf_counter()
+        R.prefill_ref(q[:1, :, t:t + 1], k[:1, :, u:u + 1], v[:1, :, u:u + 1], w.theta)
+        times.append(time.perf_counter() - a)
+        t = (t + 1) % w.h_q
+        if max_steps is not None and len(times) >= max_steps:
+            break
+        if max_steps is None and time.perf_counter() - t0 >= budget_s:
+            break
+    return per_head, times
+
+
+def cpu_baseline(w) -> dict:
+    per_head, times = oracle_prefill_sample(w, budget_s=12.0)
+    return {"value": per_head * len(times) / sum(times) / 1e12, "unit": "TFLOP/s", "cores": blas_threads(),
+            "kind": "oracle",
+            "sample": f"fp64 NumPy oracle, {len(times)} single-head slices (b=0, L={w.L}, d={w.d}) of the "
+                      f"{w.name} workload, {sum(times):.1f} s of host time"}
+
+
+def bench_config(wp, wd):
+    return {"workload": wp.desc, "B": wp.B, "L": wp.L, "h_q": wp.h_q, "h_kv": wp.h_kv, "d": wp.d,
+            "theta": wp.theta, "causal": True, "per_rank": "independent copy of the workload",
+            "l2": "flushed before every prefill (256 MiB write); decode cache 2.1 GB > L2",
+            "decode_workload": wd.desc}
+
+
+def run_reference(args):
+    rank, _, world = dist_env()
+    if rank != 0:
+        return 0
+    w = gi.BY_NAME[PREFILL_WORKLOAD]
+    per_head, times = oracle_prefill_sample(w, 0.0, max_steps=args.warmup + args.steps)
+    timed = times[args.warmup:]
+    value = per_head * len(timed) / sum(timed) / 1e12
+    line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1e3 * sum(timed) / len(timed), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": dict(bench_config(w, gi.BY_NAME[DECODE_WORKLOAD]),
+                           step="one query head of batch row 0 through the fp64 oracle on the host"),
+            "impl": "reference",
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+                             "sample": f"{len(timed)} single-head slices of {w.name}"},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------------------------------ GPU arm
+def ev():
+    e = torch.cuda.Event(enable_timing=True)
+    e.record()   # creates the CUDA event so its handle can be handed to the library
+    return e
+
+
+def run_ours(args):
+    rank, local, world = dist_env()
+    dist_init(world)
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    from grouped_query_attention_gqa_b200 import build
+    if rank == 0 or world == 1:
+        build.build()
+    barrier()
+    import grouped_query_attention_gqa_b200 as G
+    G.load()
+
+    wp = gi.BY_NAME[PREFILL_WORKLOAD]
+    wd = gi.BY_NAME[DECODE_WORKLOAD]
+    if args.decode_batch:
+        wd = wd.with_(B=args.decode_batch, desc=wd.desc.replace("B=64", f"B={args.decode_batch}"))
+    do_p, do_d = args.only in (None, "prefill"), args.only in (None, "decode")
+    q, k, v = gi.prefill_inputs(wp, device=str(dev))
+    out = torch.empty_like(q)
+    s, qd, kc, vc = gi.decode_inputs(wd, device=str(dev))
+    outd = torch.empty_like(qd)
+    total_rows = int(s.sum().item())
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    K, W = args.steps, args.warmup
+
+    def step(evs=None):
+        flush.zero_()
+        if evs:
+            evs[0].record()
+            G.set_timing_events(evs[1], evs[2])
+        if do_p:
+            G.prefill(q, k, v, theta=wp.theta, out=out)
+        if evs:
+            evs[3].record()
+            G.set_timing_events(evs[4], evs[5])
+        if do_d:
+            G.decode(qd, kc, vc, s, theta=wd.theta, out=outd)
+        if evs:
+            evs[6].record()
+            G.set_timing_events(None, None)
+
+    for _ in range(W):
+        step()
+    torch.cuda.synchronize()
+    if G.last_error() != 0:
+        raise RuntimeError("device error during warm-up")
+    evs = [[ev() for _ in range(7)] for _ in range(K)]
+    torch.cuda.synchronize()
+
+    barrier()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local)
+    with sampler:
+        t_wall = time.perf_counter()
+        for i in range(K):
+            step(evs[i])
+        torch.cuda.synchronize()
+        t_wall = time.perf_counter() - t_wall
+    barrier()
+    torch.cuda.synchronize()
+    if G.last_error() != 0:
+        raise RuntimeError("device error in the timed region")
+
+    pre_ms = [e[0].elapsed_time(e[3]) for e in evs]
+    attn_ms = [e[1].elapsed_time(e[2]) if do_p else float("nan") for e in evs]
+    dec_ms = [e[3].elapsed_time(e[6]) for e in evs]
+    split_ms = [e[4].elapsed_time(e[5]) if do_d else float("nan") for e in evs]
+    pre_mean = reduce_max(sum(pre_ms) / K, dev)
+    dec_mean = reduce_max(sum(dec_ms) / K, dev)
+    attn_mean = sum(attn_ms) / K
+    split_mean = sum(split_ms) / K
+
+    # ---- end to end through the public API: pinned host inputs in, host result out, every step
+    if not args.no_e2e:
+        qh, kh, vh = (x.cpu().pin_memory() for x in (q, k, v))
+    else:
+        qh = kh = vh = None
+    outh = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    qdh, sh_ = qd.cpu().pin_memory(), s.cpu().pin_memory()
+    outdh = torch.empty(outd.shape, dtype=outd.dtype).pin_memory()
+    qx, kx, vx, qdx, sx = (torch.empty_like(x) for x in (q, k, v, qd, s))
+
+    def e2e_step(e):
+        flush.zero_()
+        e[0].record()
+        qx.copy_(qh, non_blocking=True)
+        kx.copy_(kh, non_blocking=True)
+        vx.copy_(vh, non_blocking=True)
+        G.prefill(qx, kx, vx, theta=wp.theta, out=out)
+        outh.copy_(out, non_blocking=True)
+        e[1].record()
+        qdx.copy_(qdh, non_blocking=True)
+        sx.copy_(sh_, non_blocking=True)
+        G.decode(qdx, kc, vc, sx, theta=wd.theta, out=outd)
+        outdh.copy_(outd, non_blocking=True)
+        e[2].record()
+
+    e2e_pre = e2e_dec = float("nan")
+    if not args.no_e2e and do_p and do_d:
+        for _ in range(max(1, W)):
+            e2e_step([ev() for _ in range(3)])
+        e2e_evs = [[ev() for _ in range(3)] for _ in range(K)]
+        torch.cuda.synchronize()
+        barrier()
+        for i in range(K):
+            e2e_step(e2e_evs[i])
+        torch.cuda.synchronize()
+        barrier()
+        e2e_pre = reduce_max(sum(e[0].elapsed_time(e[1]) for e in e2e_evs) / K, dev)
+        e2e_dec = reduce_max(sum(e[1].elapsed_time(e[2]) for e in e2e_evs) / K, dev)
+
+    peaks, peak_src = load_peaks()
+    fl = prefill_flops(wp)
+    kvb = decode_kv_bytes(total_rows, wd)
+    allb = decode_bytes(total_rows, wd)
+    line = None
+    if rank == 0:
+        achieved_t = fl / (attn_mean * 1e-3) / 1e12
+        achieved_b = allb / (split_mean * 1e-3) / 1e9
+        line = {
+            "metric": METRIC,
+            "value": world * fl / (pre_mean * 1e-3) / 1e12,
+            "unit": "TFLOP/s",
+            "n_gpus": world, "steps": K, "warmup": W,
+            "ms_per_step": pre_mean,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic: seeded N(0,1) bf16 Q/K/V and caches drawn on the device; decode lengths U[1,32768]",
+            "config": bench_config(wp, wd),
+            "roofline": {"kernel": "attn_kernel (prefill)", "bound": "tensor", "achieved": achieved_t,
+                         "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved_t / peaks["bf16_tflops"],
+                         "peak_source": f"{peak_src} bf16 dense (burst)",
+                         "traffic": profile_traffic("attn_kernel_" + PREFILL_WORKLOAD),
+                         "algorithmic_flops_per_launch": fl, "ms_per_launch": attn_mean},
+            "cpu_baseline": cpu_baseline(wp) if (world == 1 and not args.no_cpu_baseline) else None,
+            "only": args.only,
+            "e2e": {"value": world * fl / (e2e_pre * 1e-3) / 1e12, "unit": "TFLOP/s",
+                    "h2d_bytes_per_step": sum(x.numel() * x.element_size() for x in (q, k, v)),
+                    "d2h_bytes_per_step": out.numel() * out.element_size()},
+            "gpu_launches": (2 * do_p + 3 * do_d) * K,
+            "clocks": sampler.summary(),
+            "decode": {
+                "workload": wd.desc, "total_cache_rows": total_rows,
+                "value": world * allb / (dec_mean * 1e-3) / 1e9, "unit": "GB/s",
+                "kv_gbs": world * kvb / (dec_mean * 1e-3) / 1e9,
+                "ms_per_step": dec_mean,
+                "roofline": {"kernel": "split_kernel (decode)", "bound": "hbm", "achieved": achieved_b,
+                             "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": achieved_b / peaks["hbm_gbs"],
+                             "peak_source": f"{peak_src} HBM copy",
+                             "traffic": profile_traffic("split_kernel_" + DECODE_WORKLOAD),
+                             "algorithmic_bytes_per_launch": allb, "ms_per_launch": split_mean},
+                "e2e": {"value": world * allb / (e2e_dec * 1e-3) / 1e9, "unit": "GB/s",
+                        "h2d_bytes_per_step": qd.numel() * 2 + s.numel() * 4,
+                        "d2h_bytes_per_step": outd.numel() * 2,
+                        "note": "the KV cache is resident device state; the step's inputs are q and the lengths"},
+            },
+            "wall_s_timed_region": t_wall,
+            "impl": "ours",
+        }
+    if torch.distributed.is_initialized():
+        barrier()
+        torch.distributed.destroy_process_group()
+    if line is not None:
+        print(json.dumps(clean(line)), flush=True)
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the host oracle timing")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffer) leg")
+    ap.add_argument("--only", choices=["prefill", "decode"], default=None,
+                    help="run one half of the step only (profiling; the line then carries that half)")
+    ap.add_argument("--decode-batch", type=int, default=None,
+                    help="decode with this many sequences instead of 64 (smaller profiling case)")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -4,5 +4,5 @@ The computation lives in libgqa.so (hand-written sm_100a CUDA behind the C ABI o
 include/gqa.h); this package is its thin Python binding.
 """
 from ._lib import (  # noqa: F401
-    GQAError, DEVERR_SEQLEN, DEVERR_TIMEOUT, LIB_PATH, decode, last_error, load, prefill, release, strerror,
+    GQAError, DEVERR_SEQLEN, DEVERR_TIMEOUT, LIB_PATH, decode, last_error, load, prefill, release, set_timing_events, strerror,
 )

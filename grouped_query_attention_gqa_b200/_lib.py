@@ -42,6 +42,8 @@ def load() -> ctypes.CDLL:
     lib.gqa_prefill.restype = i
     lib.gqa_decode.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f]
     lib.gqa_decode.restype = i
+    lib.gqa_set_timing_events.argtypes = [vp, vp]
+    lib.gqa_set_timing_events.restype = i
     lib.gqa_set_stream.argtypes = [vp]
     lib.gqa_set_stream.restype = i
     lib.gqa_last_error.argtypes = []
@@ -131,6 +133,15 @@ def last_error(device=None) -> int:
     with torch.cuda.device(dev):
         _stream(dev)
         return int(load().gqa_last_error())
+
+
+def set_timing_events(start=None, stop=None) -> None:
+    """Record torch.cuda.Event `start`/`stop` around the main kernel of later calls (None: off).
+
+    Both events must already exist on the device (record each once before handing it over).
+    """
+    h = (lambda e: None if e is None else ctypes.c_void_p(e.cuda_event))
+    load().gqa_set_timing_events(h(start), h(stop))
 
 
 def release() -> None:

@@ -32,6 +32,11 @@ struct DeviceState {
 
 DeviceState g_dev[kMaxDevices];
 cudaStream_t g_stream = nullptr;
+cudaEvent_t g_ev_start = nullptr, g_ev_stop = nullptr;   // optional timing of the main kernel
+
+inline void mark(cudaEvent_t ev) {
+    if (g_ev_start && g_ev_stop) cudaEventRecord(ev, g_stream);
+}
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                    const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -173,8 +178,10 @@ int launch_prefill(DeviceState* st, const void* q, const void* k, const void* v,
     cudaFuncAttributes fa;
     if (cudaFuncGetAttributes(&fa, attn_kernel<D>) != cudaSuccess || fa.numRegs != LAUNCH_REGS)
         return GQA_ERR_LAUNCH;
+    mark(g_ev_start);
     attn_kernel<D><<<static_cast<unsigned>(grid), NUM_THREADS, Layout<D>::DYN, g_stream>>>(tm_k, tm_v, p);
     if (cudaGetLastError() != cudaSuccess) return GQA_ERR_LAUNCH;
+    mark(g_ev_stop);
     return GQA_OK;
 }
 
@@ -214,8 +221,10 @@ int launch_decode(DeviceState* st, const void* q, const void* kc, const void* vc
     if (cudaGetLastError() != cudaSuccess) return GQA_ERR_LAUNCH;
     if (cudaFuncSetAttribute(split_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
         return GQA_ERR_LAUNCH;
+    mark(g_ev_start);
     split_kernel<D><<<G * groups, WARPS * 32, C::SMEM, g_stream>>>(p);
     if (cudaGetLastError() != cudaSuccess) return GQA_ERR_LAUNCH;
+    mark(g_ev_stop);
     const long long cgrid = static_cast<long long>(B) * groups;
     if (cgrid > 0x7fffffffLL) return GQA_ERR_DIMS;
     combine_kernel<D><<<static_cast<unsigned>(cgrid), COMBINE_THREADS, 0, g_stream>>>(p);
@@ -242,6 +251,12 @@ const char* gqa_strerror(int code) {
         case GQA_ERR_DEVICE: return "the current CUDA device is not an sm_100 GPU";
         default: return "unknown error code";
     }
+}
+
+int gqa_set_timing_events(void* start_event, void* stop_event) {
+    g_ev_start = static_cast<cudaEvent_t>(start_event);
+    g_ev_stop = static_cast<cudaEvent_t>(stop_event);
+    return GQA_OK;
 }
 
 int gqa_set_stream(void* cuda_stream) {

@@ -82,6 +82,14 @@ GQA_API int gqa_prefill(const void* q, const void* k, const void* v, void* out,
 GQA_API int gqa_decode(const void* q, const void* kcache, const void* vcache, const int* seqlens,
                void* out, int B, int h_q, int h_kv, int d, float theta);
 
+/*
+ * Measurement support.  With both events non-NULL (cudaEvent_t handles passed as void*, created
+ * by the caller), every later gqa_prefill / gqa_decode call records `start` on the current stream
+ * right before its main kernel and `stop` right after it: the attention kernel of the prefill,
+ * the split kernel of the decode.  The caller owns the events.  NULL, NULL turns this off.
+ */
+GQA_API int gqa_set_timing_events(void* start_event, void* stop_event);
+
 /* Stream for subsequent calls (a cudaStream_t passed as void*; NULL = legacy stream). */
 GQA_API int gqa_set_stream(void* cuda_stream);
 

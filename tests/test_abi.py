@@ -32,7 +32,7 @@ def codes():
 def test_header_declares_the_entry_points():
     names = set(declared())
     for n in ["gqa_prefill", "gqa_decode", "gqa_set_stream", "gqa_last_error", "gqa_release",
-              "gqa_strerror", "gqa_abi_version"]:
+              "gqa_strerror", "gqa_abi_version", "gqa_set_timing_events"]:
         assert n in names
 
 
