@@ -69,23 +69,28 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def source_sha() -> str:
-    """Hash of the library sources; a profile's DRAM traffic is used only while it matches."""
+KERNEL_SOURCES = {
+    "attn_kernel": ["prefill_sm100.cuh", "sm100_ptx.cuh", "rope.cuh"],
+    "split_kernel": ["decode_sm100.cuh", "sm100_ptx.cuh", "rope.cuh"],
+}
+
+
+def source_sha(kernel: str) -> str:
+    """Hash of the sources a kernel is built from; a profile's DRAM traffic counts only while it matches."""
     h = hashlib.sha256()
-    files = sorted(glob.glob(os.path.join(ROOT, "grouped_query_attention_gqa_b200", "csrc", "*.cu*")))
-    files.append(os.path.join(ROOT, "include", "gqa.h"))
-    for fn in files:
-        with open(fn, "rb") as f:
-            h.update(os.path.basename(fn).encode() + b"\0" + f.read())
+    for fn in KERNEL_SOURCES[kernel]:
+        with open(os.path.join(ROOT, "grouped_query_attention_gqa_b200", "csrc", fn), "rb") as f:
+            h.update(fn.encode() + b"\0" + f.read())
     return h.hexdigest()[:16]
 
 
-def profile_traffic(key: str):
-    """DRAM bytes per launch of kernel `key` from the committed ncu summaries, if still current."""
-    sha = source_sha()
+def profile_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch of `kernel` on `workload` from the committed ncu summaries, if still current."""
+    sha = source_sha(kernel)
+    key = f"{kernel}_{workload}"
     for fn in sorted(glob.glob(os.path.join(ROOT, "profiles", "*.md"))):
         txt = open(fn, encoding="utf-8").read()
-        m_sha = re.search(r"source_sha256_16:\s*([0-9a-f]{16})", txt)
+        m_sha = re.search(r"source_sha256_16\[" + kernel + r"\]:\s*([0-9a-f]{16})", txt)
         m_tr = re.search(r"traffic_bytes_per_launch\[" + re.escape(key) + r"\]:\s*([0-9.eE+]+)", txt)
         if m_sha and m_tr and m_sha.group(1) == sha:
             return float(m_tr.group(1))
@@ -390,7 +395,7 @@ def run_ours(args):
             "roofline": {"kernel": "attn_kernel (prefill)", "bound": "tensor", "achieved": achieved_t,
                          "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved_t / peaks["bf16_tflops"],
                          "peak_source": f"{peak_src} bf16 dense (burst)",
-                         "traffic": profile_traffic("attn_kernel_" + PREFILL_WORKLOAD),
+                         "traffic": profile_traffic("attn_kernel", PREFILL_WORKLOAD),
                          "algorithmic_flops_per_launch": fl, "ms_per_launch": attn_mean},
             "cpu_baseline": cpu_baseline(wp) if (world == 1 and not args.no_cpu_baseline) else None,
             "only": args.only,
@@ -407,7 +412,7 @@ def run_ours(args):
                 "roofline": {"kernel": "split_kernel (decode)", "bound": "hbm", "achieved": achieved_b,
                              "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": achieved_b / peaks["hbm_gbs"],
                              "peak_source": f"{peak_src} HBM copy",
-                             "traffic": profile_traffic("split_kernel_" + DECODE_WORKLOAD),
+                             "traffic": profile_traffic("split_kernel", DECODE_WORKLOAD),
                              "algorithmic_bytes_per_launch": allb, "ms_per_launch": split_mean},
                 "e2e": {"value": world * allb / (e2e_dec * 1e-3) / 1e9, "unit": "GB/s",
                         "h2d_bytes_per_step": qd.numel() * 2 + s.numel() * 4,
