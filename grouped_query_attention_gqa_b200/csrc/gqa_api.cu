@@ -28,6 +28,7 @@ struct DeviceState {
     size_t ws_bytes = 0;
     void* dws = nullptr;          // decode workspace
     size_t dws_bytes = 0;
+    void* fixed_scratch = nullptr;   // device address of g_fixed_scratch (gqa_decode_noalloc)
 };
 
 DeviceState g_dev[kMaxDevices];
@@ -232,6 +233,79 @@ int launch_decode(DeviceState* st, const void* q, const void* kc, const void* vc
     return GQA_OK;
 }
 
+// ---------------------------------------------------------------------------------------------
+// Decode without any device allocation (gqa_decode_noalloc).
+//
+// Who needs it: callers that own every byte of device memory themselves -- for example a serving
+// process that reserves almost all of HBM for its KV cache and model at start-up, where a cudaMalloc
+// from inside a library would fail or fragment that reservation -- and callers on a latency-critical
+// path that cannot pay for cudaMalloc / cudaFree, which may synchronise the whole device.  For them the
+// decode scratch (packed row offsets and split partials) lives in this fixed, file-scope device array,
+// which every GPU that loads the library holds until the process exits.
+constexpr size_t kFixedScratchBytes = size_t(16) << 20;   // 16 MiB per device
+static __device__ __align__(256) unsigned char g_fixed_scratch[kFixedScratchBytes];
+
+// In host code `g_fixed_scratch` names a host-side stand-in, not device memory: kernels must be given
+// the device address, looked up once per device with that device current.
+int fixed_scratch_setup(DeviceState* st) {
+    if (st->fixed_scratch) return GQA_OK;
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_fixed_scratch) != cudaSuccess || ptr == nullptr) {
+        cudaGetLastError();
+        return GQA_ERR_LAUNCH;
+    }
+    st->fixed_scratch = ptr;
+    return GQA_OK;
+}
+
+template <int D>
+int launch_decode_fixed_scratch(DeviceState* st, const void* q, const void* kc, const void* vc, const int* seqlens,
+                                void* out, int B, int h_q, int h_kv, float theta) {
+    using namespace gqa::decode;
+    using C = Cfg<D>;
+    const int g = h_q / h_kv;
+    const int n_hb = (g + HB - 1) / HB;
+    const int groups = h_kv * n_hb;
+    const int G = (2 * st->num_sms + groups - 1) / groups;
+    const int P = G * WARPS;
+    const size_t off_bytes = (static_cast<size_t>(B + 1) * sizeof(int64_t) + 255) & ~size_t(255);
+    const size_t part_bytes = static_cast<size_t>(P + B) * groups * C::PART * sizeof(float);
+    if (off_bytes + part_bytes > kFixedScratchBytes) return GQA_ERR_TOO_LARGE;
+    const int rc = fixed_scratch_setup(st);
+    if (rc != GQA_OK) return rc;
+
+    // Nothing in the scratch has to start at zero: plan_kernel rewrites all B + 1 offsets, and the
+    // combine step reads only the partials that split_kernel wrote in this same call.
+    Params p;
+    p.q = static_cast<const __nv_bfloat16*>(q);
+    p.kc = static_cast<const __nv_bfloat16*>(kc);
+    p.vc = static_cast<const __nv_bfloat16*>(vc);
+    p.out = static_cast<__nv_bfloat16*>(out);
+    p.off = static_cast<int64_t*>(st->fixed_scratch);
+    p.part = reinterpret_cast<float*>(static_cast<uint8_t*>(st->fixed_scratch) + off_bytes);
+    p.B = B;
+    p.h_q = h_q;
+    p.h_kv = h_kv;
+    p.g = g;
+    p.n_hb = n_hb;
+    p.P = P;
+    p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
+    p.theta = static_cast<double>(theta);
+    p.err = st->err;
+
+    plan_kernel<<<1, PLAN_THREADS, 0, g_stream>>>(seqlens, static_cast<int64_t*>(st->fixed_scratch), B, st->err);
+    if (cudaGetLastError() != cudaSuccess) return GQA_ERR_LAUNCH;
+    if (cudaFuncSetAttribute(split_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
+        return GQA_ERR_LAUNCH;
+    split_kernel<D><<<G * groups, WARPS * 32, C::SMEM, g_stream>>>(p);
+    if (cudaGetLastError() != cudaSuccess) return GQA_ERR_LAUNCH;
+    const long long cgrid = static_cast<long long>(B) * groups;
+    if (cgrid > 0x7fffffffLL) return GQA_ERR_DIMS;
+    combine_kernel<D><<<static_cast<unsigned>(cgrid), COMBINE_THREADS, 0, g_stream>>>(p);
+    if (cudaGetLastError() != cudaSuccess) return GQA_ERR_LAUNCH;
+    return GQA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -249,6 +323,7 @@ const char* gqa_strerror(int code) {
         case GQA_ERR_ALLOC: return "workspace allocation failed";
         case GQA_ERR_ALIGN: return "a tensor pointer is not 16-byte aligned";
         case GQA_ERR_DEVICE: return "the current CUDA device is not an sm_100 GPU";
+        case GQA_ERR_TOO_LARGE: return "the decode needs more scratch than the fixed 16 MiB buffer of gqa_decode_noalloc";
         default: return "unknown error code";
     }
 }
@@ -292,6 +367,20 @@ int gqa_decode(const void* q, const void* kcache, const void* vcache, const int*
     if (!st) return rc;
     return d == 64 ? launch_decode<64>(st, q, kcache, vcache, seqlens, out, B, h_q, h_kv, theta)
                    : launch_decode<128>(st, q, kcache, vcache, seqlens, out, B, h_q, h_kv, theta);
+}
+
+int gqa_decode_noalloc(const void* q, const void* kcache, const void* vcache, const int* seqlens, void* out, int B,
+                       int h_q, int h_kv, int d, float theta) {
+    if (B < 0) return GQA_ERR_DIMS;
+    int rc = check_common(h_q, h_kv, d, theta);
+    if (rc != GQA_OK) return rc;
+    if (B == 0) return GQA_OK;
+    if (!q || !kcache || !vcache || !seqlens || !out) return GQA_ERR_NULL;
+    if (!aligned16(q) || !aligned16(kcache) || !aligned16(vcache) || !aligned16(out)) return GQA_ERR_ALIGN;
+    DeviceState* st = device_state(&rc);
+    if (!st) return rc;
+    return d == 64 ? launch_decode_fixed_scratch<64>(st, q, kcache, vcache, seqlens, out, B, h_q, h_kv, theta)
+                   : launch_decode_fixed_scratch<128>(st, q, kcache, vcache, seqlens, out, B, h_q, h_kv, theta);
 }
 
 int gqa_last_error(void) {

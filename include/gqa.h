@@ -41,6 +41,7 @@ extern "C" {
 #define GQA_ERR_ALLOC (-6)     /* the internal workspace could not be allocated               */
 #define GQA_ERR_ALIGN (-7)     /* a tensor pointer is not 16-byte aligned                     */
 #define GQA_ERR_DEVICE (-8)    /* the current device is not an sm_100 (B200-class) GPU        */
+#define GQA_ERR_TOO_LARGE (-9) /* gqa_decode_noalloc: more scratch needed than its fixed buffer */
 
 /* Bits of the device error word returned by gqa_last_error(). */
 #define GQA_DEVERR_SEQLEN 1    /* a decode length was <= 0; that sequence's output was zeroed */
@@ -89,6 +90,33 @@ GQA_API int gqa_decode(const void* q, const void* kcache, const void* vcache, co
  * the split kernel of the decode.  The caller owns the events.  NULL, NULL turns this off.
  */
 GQA_API int gqa_set_timing_events(void* start_event, void* stop_event);
+
+/*
+ * gqa_decode_noalloc -- the same decode step as gqa_decode (same arguments, layouts, results and
+ * error codes), for callers that cannot let the library allocate device memory.  No counterpart in
+ * the paper: this is a library-level variant.
+ *
+ * Who needs it: a caller that owns all device memory itself (e.g. a serving process that reserves
+ * nearly all of HBM for its KV cache and weights up front, where a cudaMalloc from inside a library
+ * would fail or fragment that reservation), or a caller on a latency-critical path that cannot pay
+ * for cudaMalloc / cudaFree, which may synchronise the whole device.  This entry point calls no
+ * cudaMalloc, cudaFree or other allocating routine.  Its scratch (packed row offsets and split
+ * partials) is a fixed 16 MiB array in the library's device memory, which every GPU that loads the
+ * library holds until the process exits.
+ *
+ * Limit: the scratch needed is 8*(B+1) bytes rounded up to 256, plus
+ * (P + B) * h_kv * ceil(g/8) * (16 + 8*d) * 4 bytes, where P = 4 * ceil(2*SMs / (h_kv*ceil(g/8)))
+ * (P = 296 for h_kv = 4 on a 148-SM B200: the Qwen2-7B shape fits up to B of about 700).  Larger
+ * problems return GQA_ERR_TOO_LARGE and launch nothing.
+ *
+ * The first call on a device looks up the device address of the fixed array (with that device
+ * current); make that first call before any stream capture.  All calls on a device share the one
+ * array and each leaves its contents behind; nothing in it has to start at zero.  Calls whose work
+ * overlaps on the GPU (different streams, or different host threads) race on the array: serialise
+ * them on one stream.
+ */
+GQA_API int gqa_decode_noalloc(const void* q, const void* kcache, const void* vcache, const int* seqlens,
+                               void* out, int B, int h_q, int h_kv, int d, float theta);
 
 /* Stream for subsequent calls (a cudaStream_t passed as void*; NULL = legacy stream). */
 GQA_API int gqa_set_stream(void* cuda_stream);
