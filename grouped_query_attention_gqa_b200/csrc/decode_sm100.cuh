@@ -37,9 +37,16 @@ namespace decode {
 
 using namespace ptx;
 
+#ifndef GQA_DECODE_STAGES
+#define GQA_DECODE_STAGES 3
+#endif
+#ifndef GQA_DECODE_CTAS_PER_SM
+#define GQA_DECODE_CTAS_PER_SM 2
+#endif
 constexpr int ROWS = 16;        // cache rows per block (MMA M)
-constexpr int NS = 3;           // ring stages per warp
+constexpr int NS = GQA_DECODE_STAGES;             // ring stages per warp
 constexpr int WARPS = 4;        // workers per CTA
+constexpr int CTAS_PER_SM = GQA_DECODE_CTAS_PER_SM;
 constexpr int HB = 8;           // query heads per head block (MMA N)
 constexpr int REANCHOR = 64;    // blocks between exact recomputations of the RoPE angles
 constexpr int PLAN_THREADS = 1024;
@@ -55,6 +62,7 @@ struct Cfg {
     static constexpr int KS = D / 16;              // 16-wide steps along d
     static constexpr int HALF_KS = D / 32;         // steps in the first half of d
     static constexpr int NF = 4 * HALF_KS;         // RoPE frequencies owned by one lane
+    static constexpr int NP = NF / 2;              // ... as pairs of adjacent frequencies
     static constexpr int PART = 2 * HB + HB * D;   // floats per partial: m[8], l[8], O[8][D]
 };
 
@@ -165,23 +173,31 @@ struct BlockCursor {
     }
 };
 
-// Rotate the bf16 pair-halves held in x (dims i, i+1 of the first half) and y (their partners).
-__device__ __forceinline__ void rot_pair(uint32_t& x, uint32_t& y, float c0, float s0, float c1, float s1) {
-    float a0, b0, a1, b1;
-    rope_rotate(bf16lo_to_f32(x), bf16lo_to_f32(y), c0, s0, a0, b0);
-    rope_rotate(bf16hi_to_f32(x), bf16hi_to_f32(y), c1, s1, a1, b1);
-    x = pack_bf16x2(a0, a1);
-    y = pack_bf16x2(b0, b1);
+// Rotate two adjacent first-half dims (bf16x2 word x) against their partners d + D/2 (word y), with
+// (cos, sin) of the two frequencies as fp32 pairs C and S.
+__device__ __forceinline__ void rot_pair(uint32_t& x, uint32_t& y, uint64_t C, uint64_t S) {
+    const uint64_t X = f2_from_bf16x2(x), Y = f2_from_bf16x2(y);
+    x = f2_to_bf16x2(f2_sub(f2_mul(X, C), f2_mul(Y, S)));
+    y = f2_to_bf16x2(f2_fma(Y, C, f2_mul(X, S)));
+}
+
+// (C, S) <- (C, S) rotated by the angle with cosine / sine pairs (Cr, Sr): the angle-addition step.
+__device__ __forceinline__ void rot_step(uint64_t& C, uint64_t& S, uint64_t Cr, uint64_t Sr) {
+    const uint64_t c2 = f2_sub(f2_mul(C, Cr), f2_mul(S, Sr));
+    S = f2_fma(S, Cr, f2_mul(C, Sr));
+    C = c2;
 }
 
 template <int D>
-__global__ void __launch_bounds__(WARPS * 32) split_kernel(const Params p) {
+__global__ void __launch_bounds__(WARPS * 32, CTAS_PER_SM) split_kernel(const Params p) {
     using C = Cfg<D>;
     constexpr int H = D / 2;
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ uint64_t bars[WARPS][NS];
     __shared__ double finv[H];
-    __shared__ float2 rot8[H];   // cos/sin of 8 * f_i: the step between a lane's two rows of a block
+    // cos/sin of 8 * f_i for i, i+1 (i even) as {cos_i, cos_i+1, sin_i, sin_i+1}: the angle step between
+    // a lane's two rows of a block, loaded as two fp32 pairs by one 128-bit read.
+    __shared__ float4 rot8[H / 2];
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int G = gridDim.x / (p.h_kv * p.n_hb);
@@ -190,12 +206,12 @@ __global__ void __launch_bounds__(WARPS * 32) split_kernel(const Params p) {
     const int u = uh / p.n_hb, hb = uh % p.n_hb;
     const int w = gi * WARPS + warp;
 
-    for (int i = threadIdx.x; i < H; i += blockDim.x) {
-        const double f = rope_inv_freq(i, D, p.theta);
-        finv[i] = f;
-        float c, s;
-        rope_cossin(8.0, f, c, s);
-        rot8[i] = make_float2(c, s);
+    for (int i = threadIdx.x; i < H; i += blockDim.x) finv[i] = rope_inv_freq(i, D, p.theta);
+    for (int i = threadIdx.x; i < H / 2; i += blockDim.x) {
+        float c0, s0, c1, s1;
+        rope_cossin(8.0, rope_inv_freq(2 * i, D, p.theta), c0, s0);
+        rope_cossin(8.0, rope_inv_freq(2 * i + 1, D, p.theta), c1, s1);
+        rot8[i] = make_float4(c0, c1, s0, s1);
     }
     if (lane == 0) {
         for (int s = 0; s < NS; ++s) mbar_init(&bars[warp][s], 1);
@@ -266,8 +282,8 @@ __global__ void __launch_bounds__(WARPS * 32) split_kernel(const Params p) {
                 float c[4], s[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) rope_cossin(qpos, finv[d0 + (e & 1) + 8 * (e >> 1)], c[e], s[e]);
-                rot_pair(qb[ks][0], qb[ks + C::HALF_KS][0], c[0], s[0], c[1], s[1]);
-                rot_pair(qb[ks][1], qb[ks + C::HALF_KS][1], c[2], s[2], c[3], s[3]);
+                rot_pair(qb[ks][0], qb[ks + C::HALF_KS][0], f2_pack(c[0], c[1]), f2_pack(s[0], s[1]));
+                rot_pair(qb[ks][1], qb[ks + C::HALF_KS][1], f2_pack(c[2], c[3]), f2_pack(s[2], s[3]));
             }
         }
 
@@ -275,7 +291,9 @@ __global__ void __launch_bounds__(WARPS * 32) split_kernel(const Params p) {
 #pragma unroll
         for (int mt = 0; mt < C::KS; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
         float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
-        float ca[C::NF], sa[C::NF];   // cos/sin for the lane's first row of the block (row t4)
+        // cos/sin for the lane's first row of the block (row t4), as fp32 pairs of adjacent frequencies:
+        // pair 2ks holds dims 16ks + 2tq + {0, 1}, pair 2ks + 1 holds dims 16ks + 2tq + 8 + {0, 1}.
+        uint64_t ca[C::NP], sa[C::NP];
         int since_anchor = REANCHOR;
 
         while (!cur.done && cur.b == b) {
@@ -287,20 +305,24 @@ __global__ void __launch_bounds__(WARPS * 32) split_kernel(const Params p) {
 
             if (since_anchor >= REANCHOR) {
 #pragma unroll
-                for (int f = 0; f < C::NF; ++f) {
-                    const int di = 16 * (f >> 2) + 2 * tq + (f & 1) + 8 * ((f >> 1) & 1);
-                    rope_cossin(static_cast<double>(jb + t4), finv[di], ca[f], sa[f]);
+                for (int fp = 0; fp < C::NP; ++fp) {
+                    const int di = 16 * (fp >> 1) + 2 * tq + 8 * (fp & 1);
+                    float c0, s0, c1, s1;
+                    rope_cossin(static_cast<double>(jb + t4), finv[di], c0, s0);
+                    rope_cossin(static_cast<double>(jb + t4), finv[di + 1], c1, s1);
+                    ca[fp] = f2_pack(c0, c1);
+                    sa[fp] = f2_pack(s0, s1);
                 }
                 since_anchor = 0;
             }
             // cos/sin for row t4 + 8
-            float cb[C::NF], sb[C::NF];
+            uint64_t cb[C::NP], sb[C::NP];
 #pragma unroll
-            for (int f = 0; f < C::NF; ++f) {
-                const int di = 16 * (f >> 2) + 2 * tq + (f & 1) + 8 * ((f >> 1) & 1);
-                const float2 r8 = rot8[di];
-                cb[f] = fmaf(ca[f], r8.x, -sa[f] * r8.y);
-                sb[f] = fmaf(sa[f], r8.x, ca[f] * r8.y);
+            for (int fp = 0; fp < C::NP; ++fp) {
+                const float4 r8 = rot8[(16 * (fp >> 1) + 2 * tq + 8 * (fp & 1)) >> 1];
+                cb[fp] = ca[fp];
+                sb[fp] = sa[fp];
+                rot_step(cb[fp], sb[fp], f2_pack(r8.x, r8.y), f2_pack(r8.z, r8.w));
             }
 
             const uint32_t k_a = wsm_a + stage * C::STAGE;
@@ -313,21 +335,20 @@ __global__ void __launch_bounds__(WARPS * 32) split_kernel(const Params p) {
                 uint32_t a[4], a2[4];
                 ldsm_x4(krow + 16 * ks * 2, a[0], a[1], a[2], a[3]);
                 ldsm_x4(krow + 16 * (ks + C::HALF_KS) * 2, a2[0], a2[1], a2[2], a2[3]);
-                const int f = 4 * ks;
-                rot_pair(a[0], a2[0], ca[f], sa[f], ca[f + 1], sa[f + 1]);           // row t4,   dims +0,+1
-                rot_pair(a[1], a2[1], cb[f], sb[f], cb[f + 1], sb[f + 1]);           // row t4+8, dims +0,+1
-                rot_pair(a[2], a2[2], ca[f + 2], sa[f + 2], ca[f + 3], sa[f + 3]);   // row t4,   dims +8,+9
-                rot_pair(a[3], a2[3], cb[f + 2], sb[f + 2], cb[f + 3], sb[f + 3]);   // row t4+8, dims +8,+9
+                rot_pair(a[0], a2[0], ca[2 * ks], sa[2 * ks]);           // row t4,   dims +0,+1
+                rot_pair(a[1], a2[1], cb[2 * ks], sb[2 * ks]);           // row t4+8, dims +0,+1
+                rot_pair(a[2], a2[2], ca[2 * ks + 1], sa[2 * ks + 1]);   // row t4,   dims +8,+9
+                rot_pair(a[3], a2[3], cb[2 * ks + 1], sb[2 * ks + 1]);   // row t4+8, dims +8,+9
                 mma_bf16_16816(sacc, a[0], a[1], a[2], a[3], qb[ks][0], qb[ks][1]);
                 mma_bf16_16816(sacc, a2[0], a2[1], a2[2], a2[3], qb[ks + C::HALF_KS][0], qb[ks + C::HALF_KS][1]);
             }
             // advance the angles to the next block's first row (row t4 + 16)
 #pragma unroll
-            for (int f = 0; f < C::NF; ++f) {
-                const int di = 16 * (f >> 2) + 2 * tq + (f & 1) + 8 * ((f >> 1) & 1);
-                const float2 r8 = rot8[di];
-                ca[f] = fmaf(cb[f], r8.x, -sb[f] * r8.y);
-                sa[f] = fmaf(sb[f], r8.x, cb[f] * r8.y);
+            for (int fp = 0; fp < C::NP; ++fp) {
+                const float4 r8 = rot8[(16 * (fp >> 1) + 2 * tq + 8 * (fp & 1)) >> 1];
+                ca[fp] = cb[fp];
+                sa[fp] = sb[fp];
+                rot_step(ca[fp], sa[fp], f2_pack(r8.x, r8.y), f2_pack(r8.z, r8.w));
             }
             ++since_anchor;
 
@@ -397,10 +418,22 @@ __global__ void __launch_bounds__(WARPS * 32) split_kernel(const Params p) {
 }
 
 // ---------------------------------------------------------------------------------------------
+// One CTA per (sequence, KV group, head block).  The pieces of the sequence are processed CHUNK at a
+// time: one thread per piece reads its (m, l) for the 8 heads, warp h reduces head h over the chunk
+// (max, then the rescaled sum), and each thread accumulates 4 of the 8 x D outputs over the pieces with
+// several loads in flight.
 template <int D>
 __global__ void __launch_bounds__(COMBINE_THREADS) combine_kernel(const Params p) {
     using C = Cfg<D>;
-    __shared__ float sM[HB], sInvL[HB];
+    constexpr int CHUNK = COMBINE_THREADS;   // pieces per round
+    constexpr int PER_T = HB * D / COMBINE_THREADS;
+    static_assert(COMBINE_THREADS == 32 * HB, "one warp per head");
+    static_assert(HB * D % COMBINE_THREADS == 0, "outputs split evenly");
+    __shared__ float s_m[CHUNK][HB + 1];
+    __shared__ float s_l[CHUNK][HB + 1];
+    __shared__ const float* s_ptr[CHUNK];
+    __shared__ float s_M[HB], s_L[HB];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int hb = blockIdx.x % p.n_hb;
     const int u = (blockIdx.x / p.n_hb) % p.h_kv;
     const int b = blockIdx.x / (p.n_hb * p.h_kv);
@@ -409,40 +442,75 @@ __global__ void __launch_bounds__(COMBINE_THREADS) combine_kernel(const Params p
     const int64_t s0 = p.off[b], s1 = p.off[b + 1];
     __nv_bfloat16* ob = p.out + (static_cast<int64_t>(b) * p.h_q + u * p.g + hb * HB) * D;
     if (s1 <= s0) {   // empty (invalid) sequence: zeros, flagged by plan_kernel
-        for (int e = threadIdx.x; e < nh * D; e += blockDim.x) ob[e] = __float2bfloat16(0.f);
+        for (int e = tid; e < nh * D; e += blockDim.x) ob[e] = __float2bfloat16(0.f);
         return;
     }
     const int w_lo = slice_of(s0, N, p.P);
     const int w_hi = slice_of(s1 - 1, N, p.P);
-    auto part_of = [&](int w) {
-        return p.part + ((static_cast<int64_t>(w + b) * p.h_kv + u) * p.n_hb + hb) * C::PART;
-    };
-    // Slices strictly inside (w_lo, w_hi) may be empty when N < P: they wrote nothing.
-    auto empty = [&](int w) { return slice_start(N, w + 1, p.P) <= slice_start(N, w, p.P); };
-    if (threadIdx.x < nh) {
-        const int h = threadIdx.x;
-        float M = -INFINITY;
-        for (int w = w_lo; w <= w_hi; ++w)
-            if (!empty(w)) M = fmaxf(M, part_of(w)[h]);
-        float L = 0.f;
-        for (int w = w_lo; w <= w_hi; ++w) {
-            if (empty(w)) continue;
-            const float* pp = part_of(w);
-            L += pp[HB + h] * ex2(pp[h] - M);
+    // Pass 1: merged max M and sum L per head.  Slices strictly inside (w_lo, w_hi) may be empty when
+    // N < P: they wrote nothing and are skipped.
+    float M = -INFINITY, L = 0.f;   // warp `warp` tracks head `warp`
+    for (int w0 = w_lo; w0 <= w_hi; w0 += CHUNK) {
+        const int w = w0 + tid;
+        const bool live = w <= w_hi && slice_start(N, w + 1, p.P) > slice_start(N, w, p.P);
+        const float* pp = live ? p.part + ((static_cast<int64_t>(w + b) * p.h_kv + u) * p.n_hb + hb) * C::PART
+                               : nullptr;
+        s_ptr[tid] = pp;
+#pragma unroll
+        for (int h = 0; h < HB; ++h) {
+            s_m[tid][h] = live ? pp[h] : -INFINITY;
+            s_l[tid][h] = live ? pp[HB + h] : 0.f;
         }
-        sM[h] = M;
-        sInvL[h] = 1.0f / L;
+        __syncthreads();
+        float m = -INFINITY;
+        for (int i = lane; i < CHUNK; i += 32) m = fmaxf(m, s_m[i][warp]);
+#pragma unroll
+        for (int sh = 16; sh > 0; sh >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, sh));
+        const float Mn = fmaxf(M, m);
+        float l = 0.f;
+        for (int i = lane; i < CHUNK; i += 32) l += s_l[i][warp] * ex2(s_m[i][warp] - Mn);
+#pragma unroll
+        for (int sh = 16; sh > 0; sh >>= 1) l += __shfl_xor_sync(0xffffffffu, l, sh);
+        L = L * ex2(M - Mn) + l;
+        M = Mn;
+        __syncthreads();
+    }
+    if (lane == 0) {
+        s_M[warp] = M;
+        s_L[warp] = L;
     }
     __syncthreads();
-    for (int e = threadIdx.x; e < nh * D; e += blockDim.x) {
-        const int h = e / D, d = e % D;
-        float acc = 0.f;
-        for (int w = w_lo; w <= w_hi; ++w) {
-            if (empty(w)) continue;
-            const float* pp = part_of(w);
-            acc += pp[2 * HB + h * D + d] * ex2(pp[h] - sM[h]);
+    // Pass 2: O = sum over pieces of O_piece * 2^(m_piece - M) / L.
+    float acc[PER_T];
+#pragma unroll
+    for (int k = 0; k < PER_T; ++k) acc[k] = 0.f;
+    for (int w0 = w_lo; w0 <= w_hi; w0 += CHUNK) {
+        const int w = w0 + tid;
+        const bool live = w <= w_hi && slice_start(N, w + 1, p.P) > slice_start(N, w, p.P);
+        const float* pp = live ? p.part + ((static_cast<int64_t>(w + b) * p.h_kv + u) * p.n_hb + hb) * C::PART
+                               : nullptr;
+        s_ptr[tid] = pp;
+#pragma unroll
+        for (int h = 0; h < HB; ++h) s_m[tid][h] = live ? ex2(pp[h] - s_M[h]) / s_L[h] : 0.f;   // weights
+        __syncthreads();
+        const int n = min(CHUNK, w_hi - w0 + 1);
+#pragma unroll 4
+        for (int i = 0; i < n; ++i) {
+            const float* po = s_ptr[i];
+            if (po == nullptr) continue;
+            po += 2 * HB;
+#pragma unroll
+            for (int k = 0; k < PER_T; ++k) {
+                const int e = tid + k * COMBINE_THREADS;
+                acc[k] = fmaf(po[e], s_m[i][e / D], acc[k]);
+            }
         }
-        ob[e] = __float2bfloat16(acc * sInvL[h]);
+        __syncthreads();
+    }
+#pragma unroll
+    for (int k = 0; k < PER_T; ++k) {
+        const int e = tid + k * COMBINE_THREADS;
+        if (e < nh * D) ob[e] = __float2bfloat16(acc[k]);
     }
 }
 

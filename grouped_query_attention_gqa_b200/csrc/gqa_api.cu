@@ -126,40 +126,51 @@ template <int D>
 int launch_prefill(DeviceState* st, const void* q, const void* k, const void* v, void* out, int B, int L, int h_q,
                    int h_kv, float theta) {
     using namespace gqa::prefill;
+    // Workspace: Q' [B*h_q, L, D] then K' [B*h_kv, L, D], both bf16, rotated.
+    const size_t qr_bytes = (static_cast<size_t>(B) * h_q * L * D * 2 + 255) & ~size_t(255);
     const size_t kr_bytes = static_cast<size_t>(B) * h_kv * L * D * 2;
-    const size_t cs_off = (kr_bytes + 255) & ~size_t(255);
-    const size_t need = cs_off + static_cast<size_t>(L) * (D / 2) * sizeof(float2);
-    if (!ensure(st->ws, st->ws_bytes, need)) return GQA_ERR_ALLOC;
-    auto* kr = static_cast<__nv_bfloat16*>(st->ws);
-    auto* cs = reinterpret_cast<float2*>(static_cast<uint8_t*>(st->ws) + cs_off);
+    if (!ensure(st->ws, st->ws_bytes, qr_bytes + kr_bytes)) return GQA_ERR_ALLOC;
+    auto* qr = static_cast<__nv_bfloat16*>(st->ws);
+    auto* kr = reinterpret_cast<__nv_bfloat16*>(static_cast<uint8_t*>(st->ws) + qr_bytes);
 
     if (!get_encoder()) return GQA_ERR_LAUNCH;
-    CUtensorMap tm_k, tm_v;
+    CUtensorMap tm_q, tm_k, tm_v, tm_o;
+    const cuuint32_t box3[3] = {64, BM, 1};
+    {   // Q' [B*h_q, L, D]
+        const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(L),
+                                    static_cast<cuuint64_t>(B) * h_q};
+        const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(L) * D * 2};
+        if (!encode_bf16(&tm_q, qr, 3, dims, strides, box3)) return GQA_ERR_LAUNCH;
+    }
     {   // K' [B*h_kv, L, D]
         const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(L),
                                     static_cast<cuuint64_t>(B) * h_kv};
         const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(L) * D * 2};
-        const cuuint32_t box[3] = {64, BN, 1};
-        if (!encode_bf16(&tm_k, kr, 3, dims, strides, box)) return GQA_ERR_LAUNCH;
+        if (!encode_bf16(&tm_k, kr, 3, dims, strides, box3)) return GQA_ERR_LAUNCH;
     }
-    {   // V [B, L, h_kv, D]
+    const cuuint32_t box4[4] = {64, 1, BN, 1};
+    {   // V [B, L, h_kv, D], read in place
         const cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(h_kv),
                                     static_cast<cuuint64_t>(L), static_cast<cuuint64_t>(B)};
         const cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(h_kv) * D * 2,
                                        static_cast<cuuint64_t>(L) * h_kv * D * 2};
-        const cuuint32_t box[4] = {64, 1, BN, 1};
-        if (!encode_bf16(&tm_v, v, 4, dims, strides, box)) return GQA_ERR_LAUNCH;
+        if (!encode_bf16(&tm_v, v, 4, dims, strides, box4)) return GQA_ERR_LAUNCH;
+    }
+    {   // out [B, L, h_q, D], written by TMA stores
+        const cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(h_q),
+                                    static_cast<cuuint64_t>(L), static_cast<cuuint64_t>(B)};
+        const cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(h_q) * D * 2,
+                                       static_cast<cuuint64_t>(L) * h_q * D * 2};
+        if (!encode_bf16(&tm_o, out, 4, dims, strides, box4)) return GQA_ERR_LAUNCH;
     }
 
     const int prep_blocks = (L + PREP_POS - 1) / PREP_POS;
-    prep_kernel<D><<<prep_blocks, PREP_THREADS, 0, g_stream>>>(static_cast<const __nv_bfloat16*>(k), kr, cs, B, L,
-                                                               h_kv, static_cast<double>(theta));
+    prep_kernel<D><<<prep_blocks, PREP_THREADS, 0, g_stream>>>(static_cast<const __nv_bfloat16*>(q),
+                                                               static_cast<const __nv_bfloat16*>(k), qr, kr, B, L,
+                                                               h_q, h_kv, static_cast<double>(theta));
     if (cudaGetLastError() != cudaSuccess) return GQA_ERR_LAUNCH;
 
     Params p;
-    p.q = static_cast<const __nv_bfloat16*>(q);
-    p.out = static_cast<__nv_bfloat16*>(out);
-    p.cs = cs;
     p.B = B;
     p.L = L;
     p.h_q = h_q;
@@ -180,7 +191,7 @@ int launch_prefill(DeviceState* st, const void* q, const void* k, const void* v,
     if (cudaFuncGetAttributes(&fa, attn_kernel<D>) != cudaSuccess || fa.numRegs != LAUNCH_REGS)
         return GQA_ERR_LAUNCH;
     mark(g_ev_start);
-    attn_kernel<D><<<static_cast<unsigned>(grid), NUM_THREADS, Layout<D>::DYN, g_stream>>>(tm_k, tm_v, p);
+    attn_kernel<D><<<static_cast<unsigned>(grid), NUM_THREADS, Layout<D>::DYN, g_stream>>>(tm_q, tm_k, tm_v, tm_o, p);
     if (cudaGetLastError() != cudaSuccess) return GQA_ERR_LAUNCH;
     mark(g_ev_stop);
     return GQA_OK;
@@ -194,8 +205,8 @@ int launch_decode(DeviceState* st, const void* q, const void* kc, const void* vc
     const int g = h_q / h_kv;
     const int n_hb = (g + HB - 1) / HB;
     const int groups = h_kv * n_hb;
-    // About two CTAs of WARPS workers per SM in total, split evenly over the (group, head block) pairs.
-    const int G = (2 * st->num_sms + groups - 1) / groups;
+    // CTAS_PER_SM CTAs of WARPS workers per SM in total, split evenly over the (group, head block) pairs.
+    const int G = (CTAS_PER_SM * st->num_sms + groups - 1) / groups;
     const int P = G * WARPS;
     const size_t off_bytes = (static_cast<size_t>(B + 1) * sizeof(int64_t) + 255) & ~size_t(255);
     const size_t part_bytes = static_cast<size_t>(P + B) * groups * C::PART * sizeof(float);
@@ -266,7 +277,7 @@ int launch_decode_fixed_scratch(DeviceState* st, const void* q, const void* kc, 
     const int g = h_q / h_kv;
     const int n_hb = (g + HB - 1) / HB;
     const int groups = h_kv * n_hb;
-    const int G = (2 * st->num_sms + groups - 1) / groups;
+    const int G = (CTAS_PER_SM * st->num_sms + groups - 1) / groups;
     const int P = G * WARPS;
     const size_t off_bytes = (static_cast<size_t>(B + 1) * sizeof(int64_t) + 255) & ~size_t(255);
     const size_t part_bytes = static_cast<size_t>(P + B) * groups * C::PART * sizeof(float);
@@ -348,7 +359,8 @@ int gqa_prefill(const void* q, const void* k, const void* v, void* out, int B, i
     if (!q || !k || !v || !out) return GQA_ERR_NULL;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return GQA_ERR_ALIGN;
     // TMA coordinates are 32-bit and the kernel indexes rows with 32-bit positions.
-    if (static_cast<long long>(B) * h_kv > 0x7fffffffLL || L > (1 << 30)) return GQA_ERR_DIMS;
+    // TMA coordinates are 32-bit; the prep kernel indexes B * (h_q + h_kv) * 8 * d / 16 items in 32 bits.
+    if (static_cast<long long>(B) * (h_q + h_kv) * 64 > 0x7fffffffLL || L > (1 << 30)) return GQA_ERR_DIMS;
     DeviceState* st = device_state(&rc);
     if (!st) return rc;
     return d == 64 ? launch_prefill<64>(st, q, k, v, out, B, L, h_q, h_kv, theta)

@@ -8,15 +8,16 @@
 // §4.1.3 step 5).  Q' and K' are the RoPE-rotated rows (rope.cuh).
 //
 // Two kernels:
-//  * prep_kernel: one cos/sin table [L, d/2] shared by Q and K, and K rotated
-//    once into a head-major buffer K' [B, h_kv, L, d].  Every K' tile is then
-//    read by ~L/256 * g query tiles, so rotating it once beats rotating it on
-//    every use.
-//  * attn_kernel: one CTA per pair of 128-row query tiles of the same
-//    (b, KV group); each K'/V tile is brought into shared memory once by TMA
-//    and consumed by both tiles (GQA reuse inside the CTA; the remaining heads
-//    of the group hit the same tiles in L2).  Q is rotated in registers on its
-//    way into shared memory.
+//  * prep_kernel: Q and K rotated once, into head-major buffers Q' [B, h_q, L, d] and
+//    K' [B, h_kv, L, d], with one cos/sin table per block of positions shared by Q and K (page
+//    "Qwen2 / Qwen3 的实测配置差异与三个坑", docs.keinmal.top, closing note of pitfall 3).  It is a
+//    streaming, bandwidth-bound pass; rotating there instead of in the attention kernel takes the
+//    rotation (and its latency) off the start of every attention CTA, and every K' tile is read by
+//    ~L/256 * g query tiles, so rotating K once beats rotating it on each use.
+//  * attn_kernel: one CTA per pair of 128-row query tiles of the same (b, KV group); Q', K' and V
+//    tiles arrive by TMA; each K'/V tile is brought into shared memory once and consumed by both
+//    query tiles (GQA reuse inside the CTA; the remaining heads of the group hit the same tiles in
+//    L2).  The output tile is staged in the (by then idle) Q' tile and written by a TMA store.
 //
 // Warp roles (384 threads, three warpgroups):
 //   warps 0-3  softmax for query tile 0   (thread = query row = TMEM lane)
@@ -60,13 +61,20 @@ constexpr int OTHER_REGS = 56;
 static_assert(256 * SOFTMAX_REGS + 128 * OTHER_REGS == NUM_THREADS * LAUNCH_REGS, "register split");
 constexpr uint32_t TMEM_COLS = 512;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: O is rescaled only when the max grows by > 2^8
-constexpr int PREP_POS = 32;                // positions per CTA of the prep kernel
+// Of every 8 consecutive exponentials of a row (off the diagonal tile), this many run on the FMA
+// pipe (exp2_poly) and the rest on the ex2 unit.
+#ifndef GQA_EXP_POLY_OF_8
+#define GQA_EXP_POLY_OF_8 0
+#endif
+// 1: round P to bf16 with integer ops instead of the conversion instruction.
+#ifndef GQA_PACK_INT
+#define GQA_PACK_INT 0
+#endif
+constexpr int PREP_POS = 8;                 // positions per CTA of the prep kernel
+constexpr int PREP_UNROLL = 4;              // work items per thread in flight
 constexpr int PREP_THREADS = 256;
 
 struct Params {
-    const __nv_bfloat16* q;    // [B, L, h_q, D]
-    __nv_bfloat16* out;        // [B, L, h_q, D]
-    const float2* cs;          // [L, D/2]  (cos, sin) of position * theta^(-2i/D)
     int B, L, h_q, h_kv, g;
     int n_qtiles;              // ceil(L / BM)
     int tiles_per_group;       // n_qtiles * g
@@ -97,63 +105,120 @@ struct alignas(8) Shared {
 };
 
 // ---------------------------------------------------------------------------------------------
-// prep_kernel: cos/sin table for positions [p0, p0+PREP_POS) and K' for those positions.
+// prep_kernel: for positions [p0, p0+PREP_POS): the cos/sin table, then every Q and K row at those
+// positions rotated into Q' [B*h_q, L, D] and K' [B*h_kv, L, D].
 template <int D>
-__global__ void __launch_bounds__(PREP_THREADS) prep_kernel(const __nv_bfloat16* __restrict__ k,
-                                                            __nv_bfloat16* __restrict__ kr,
-                                                            float2* __restrict__ cs, int B, int L,
-                                                            int h_kv, double theta) {
+__global__ void __launch_bounds__(PREP_THREADS) prep_kernel(const __nv_bfloat16* __restrict__ q,
+                                                            const __nv_bfloat16* __restrict__ k,
+                                                            __nv_bfloat16* __restrict__ qr,
+                                                            __nv_bfloat16* __restrict__ kr, int B, int L,
+                                                            int h_q, int h_kv, double theta) {
     constexpr int H = D / 2;
+    constexpr int CH = D / 16;   // one work item = 8 pairs: a 16-byte chunk of the first half + its partner
     __shared__ float2 tab[PREP_POS][H];
     __shared__ double finv[H];
     const int p0 = blockIdx.x * PREP_POS;
+    const int heads = h_q + h_kv;
+    const int items = B * heads * PREP_POS * CH;   // < 2^31: B * (h_q + h_kv) is checked on the host
+
+    // PREP_UNROLL items per thread per round, loads first, so each thread keeps several 32-byte reads in
+    // flight (the pass is bandwidth bound); the first round's loads are issued before the table is built.
+    uint4 x[PREP_UNROLL], y[PREP_UNROLL];
+    __nv_bfloat16* dst[PREP_UNROLL];
+    int cc[PREP_UNROLL], ppp[PREP_UNROLL];
+    auto load_round = [&](int base) {
+#pragma unroll
+        for (int uidx = 0; uidx < PREP_UNROLL; ++uidx) {
+            const int e = base + uidx * static_cast<int>(blockDim.x);
+            dst[uidx] = nullptr;
+            cc[uidx] = e % CH;
+            ppp[uidx] = (e / CH) % PREP_POS;
+            const int bh = e / (CH * PREP_POS);
+            const int pos = p0 + ppp[uidx];
+            if (e >= items || pos >= L) continue;
+            const int b = bh / heads, h = bh % heads;
+            const __nv_bfloat16* src;
+            if (h < h_q) {
+                src = q + ((static_cast<int64_t>(b) * L + pos) * h_q + h) * D;
+                dst[uidx] = qr + ((static_cast<int64_t>(b) * h_q + h) * L + pos) * D;
+            } else {
+                src = k + ((static_cast<int64_t>(b) * L + pos) * h_kv + (h - h_q)) * D;
+                dst[uidx] = kr + ((static_cast<int64_t>(b) * h_kv + (h - h_q)) * L + pos) * D;
+            }
+            x[uidx] = __ldg(reinterpret_cast<const uint4*>(src) + cc[uidx]);
+            y[uidx] = __ldg(reinterpret_cast<const uint4*>(src) + cc[uidx] + CH);
+        }
+    };
+    int base = threadIdx.x;
+    load_round(base);
+
     for (int i = threadIdx.x; i < H; i += blockDim.x) finv[i] = rope_inv_freq(i, D, theta);
     __syncthreads();
     for (int e = threadIdx.x; e < PREP_POS * H; e += blockDim.x) {
         const int pp = e / H, i = e % H;
-        const int pos = p0 + pp;
-        if (pos < L) {
-            float c, s;
-            rope_cossin(static_cast<double>(pos), finv[i], c, s);
-            tab[pp][i] = make_float2(c, s);
-            cs[static_cast<size_t>(pos) * H + i] = make_float2(c, s);
-        }
+        float c = 1.f, s = 0.f;
+        if (p0 + pp < L) rope_cossin(static_cast<double>(p0 + pp), finv[i], c, s);
+        tab[pp][i] = make_float2(c, s);
     }
     __syncthreads();
-    // One work item = 8 pairs (16-byte chunk of the first half + its partner chunk).
-    constexpr int CH = D / 16;
-    const int64_t items = static_cast<int64_t>(PREP_POS) * B * h_kv * CH;
-    for (int64_t e = threadIdx.x; e < items; e += blockDim.x) {
-        const int c = static_cast<int>(e % CH);
-        const int64_t rr = e / CH;
-        const int pp = static_cast<int>(rr % PREP_POS);
-        const int64_t bu = rr / PREP_POS;
-        const int b = static_cast<int>(bu / h_kv), u = static_cast<int>(bu % h_kv);
-        const int pos = p0 + pp;
-        if (pos >= L) continue;
-        const uint4* src = reinterpret_cast<const uint4*>(k + ((static_cast<int64_t>(b) * L + pos) * h_kv + u) * D);
-        uint4* dst = reinterpret_cast<uint4*>(kr + ((static_cast<int64_t>(b) * h_kv + u) * L + pos) * D);
-        const uint4 x = __ldg(src + c);
-        const uint4 y = __ldg(src + c + CH);
-        const uint32_t xs[4] = {x.x, x.y, x.z, x.w};
-        const uint32_t ys[4] = {y.x, y.y, y.z, y.w};
-        uint32_t xo[4], yo[4];
+
+    for (; base < items; base += PREP_UNROLL * static_cast<int>(blockDim.x)) {
+        if (base != threadIdx.x) load_round(base);
 #pragma unroll
-        for (int w = 0; w < 4; ++w) {
-            const float2 c0 = tab[pp][8 * c + 2 * w];
-            const float2 c1 = tab[pp][8 * c + 2 * w + 1];
-            float a0, b0, a1, b1;
-            rope_rotate(bf16lo_to_f32(xs[w]), bf16lo_to_f32(ys[w]), c0.x, c0.y, a0, b0);
-            rope_rotate(bf16hi_to_f32(xs[w]), bf16hi_to_f32(ys[w]), c1.x, c1.y, a1, b1);
-            xo[w] = pack_bf16x2(a0, a1);
-            yo[w] = pack_bf16x2(b0, b1);
+        for (int uidx = 0; uidx < PREP_UNROLL; ++uidx) {
+            if (dst[uidx] == nullptr) continue;
+            const int c = cc[uidx], pp = ppp[uidx];
+            const uint32_t xs[4] = {x[uidx].x, x[uidx].y, x[uidx].z, x[uidx].w};
+            const uint32_t ys[4] = {y[uidx].x, y[uidx].y, y[uidx].z, y[uidx].w};
+            uint32_t xo[4], yo[4];
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+                const float2 c0 = tab[pp][8 * c + 2 * w];
+                const float2 c1 = tab[pp][8 * c + 2 * w + 1];
+                float a0, b0, a1, b1;
+                rope_rotate(bf16lo_to_f32(xs[w]), bf16lo_to_f32(ys[w]), c0.x, c0.y, a0, b0);
+                rope_rotate(bf16hi_to_f32(xs[w]), bf16hi_to_f32(ys[w]), c1.x, c1.y, a1, b1);
+                xo[w] = pack_bf16x2(a0, a1);
+                yo[w] = pack_bf16x2(b0, b1);
+            }
+            reinterpret_cast<uint4*>(dst[uidx])[c] = make_uint4(xo[0], xo[1], xo[2], xo[3]);
+            reinterpret_cast<uint4*>(dst[uidx])[c + CH] = make_uint4(yo[0], yo[1], yo[2], yo[3]);
         }
-        dst[c] = make_uint4(xo[0], xo[1], xo[2], xo[3]);
-        dst[c + CH] = make_uint4(yo[0], yo[1], yo[2], yo[3]);
     }
 }
 
-// ---------------------------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t pack_p(float lo, float hi) {
+#if GQA_PACK_INT
+    return pack_bf16x2_int(lo, hi);
+#else
+    return pack_bf16x2(lo, hi);
+#endif
+}
+
+// P = 2^(s * scale_log2 - m) for one row of 128 scores, stored as bf16 pairs into the first 64
+// columns of the S region (chunk c overwrites S columns 16c.., already in registers); returns the
+// row sum of the fp32 values.  POLY: part of the exponentials on the FMA pipe (never on a tile
+// with masked entries, whose weights must be exactly 0).
+template <bool POLY>
+__device__ __forceinline__ float row_exp_store(const uint32_t (&sr)[4][32], float sl2, float neg_m, uint32_t t_s) {
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+            const float x0 = fmaf(__uint_as_float(sr[c][e]), sl2, neg_m);
+            const float x1 = fmaf(__uint_as_float(sr[c][e + 1]), sl2, neg_m);
+            const float p0 = (POLY && (e & 7) < GQA_EXP_POLY_OF_8) ? exp2_poly(x0) : ex2(x0);
+            const float p1 = (POLY && ((e + 1) & 7) < GQA_EXP_POLY_OF_8) ? exp2_poly(x1) : ex2(x1);
+            acc[(e >> 1) & 3] += p0 + p1;
+            pk[e >> 1] = pack_p(p0, p1);
+        }
+        tmem_st16(t_s + 16 * c, pk);
+    }
+    return (acc[0] + acc[1]) + (acc[2] + acc[3]);
+}
+
 // Byte address of 16-byte chunk `cc` (8 bf16 along d) of row r in a K-major, 128-byte-swizzled tile.
 __device__ __forceinline__ uint32_t swz_off(int r, int cc) {
     return static_cast<uint32_t>((cc >> 3) * (BM * 128) + r * 128 + (((cc & 7) ^ (r & 7)) << 4));
@@ -161,7 +226,8 @@ __device__ __forceinline__ uint32_t swz_off(int r, int cc) {
 
 template <int D>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
-    attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+    attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
                 const Params p) {
     using Lay = Layout<D>;
     extern __shared__ uint8_t dyn_smem_raw[];
@@ -184,8 +250,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int nmax = n0 > n1 ? n0 : n1;
 
     if (threadIdx.x == 0) {
-        mbar_init(&sh.q_full[0], 128);
-        mbar_init(&sh.q_full[1], 128);
+        mbar_init(&sh.q_full[0], 1);
+        mbar_init(&sh.q_full[1], 1);
         for (int s = 0; s < KSTAGES; ++s) {
             mbar_init(&sh.k_full[s], 1);
             mbar_init(&sh.k_empty[s], 1);
@@ -208,8 +274,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tmem_relinquish();
     }
     if (warp == WARP_TMA && lane == 0) {
+        prefetch_tensormap(&tm_q);
         prefetch_tensormap(&tm_k);
         prefetch_tensormap(&tm_v);
+        prefetch_tensormap(&tm_o);
     }
     tc_fence_before();
     __syncthreads();
@@ -229,39 +297,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int qtk = nk - 1;
         const int headk = u * p.g + idx % p.g;
         if (nk > 0) {
-            const int row = qtk * BM + r;
-            // ---- Q: load, rotate at position `row`, store bf16 into the swizzled tile.
-            uint8_t* qs = smem + Lay::Q0 + k * Lay::TILE;
-            constexpr int CH = D / 16;
-            if (row < p.L) {
-                const uint4* src = reinterpret_cast<const uint4*>(
-                    p.q + ((static_cast<int64_t>(b) * p.L + row) * p.h_q + headk) * D);
-                const float4* csr = reinterpret_cast<const float4*>(p.cs + static_cast<int64_t>(row) * (D / 2));
-#pragma unroll
-                for (int c = 0; c < CH; ++c) {
-                    const uint4 x = __ldg(src + c);
-                    const uint4 y = __ldg(src + c + CH);
-                    const uint32_t xs[4] = {x.x, x.y, x.z, x.w};
-                    const uint32_t ys[4] = {y.x, y.y, y.z, y.w};
-                    uint32_t xo[4], yo[4];
-#pragma unroll
-                    for (int w = 0; w < 4; ++w) {
-                        const float4 t2 = __ldg(csr + 4 * c + w);   // (cos, sin) for pairs 8c+2w, 8c+2w+1
-                        float a0, b0, a1, b1;
-                        rope_rotate(bf16lo_to_f32(xs[w]), bf16lo_to_f32(ys[w]), t2.x, t2.y, a0, b0);
-                        rope_rotate(bf16hi_to_f32(xs[w]), bf16hi_to_f32(ys[w]), t2.z, t2.w, a1, b1);
-                        xo[w] = pack_bf16x2(a0, a1);
-                        yo[w] = pack_bf16x2(b0, b1);
-                    }
-                    *reinterpret_cast<uint4*>(qs + swz_off(r, c)) = make_uint4(xo[0], xo[1], xo[2], xo[3]);
-                    *reinterpret_cast<uint4*>(qs + swz_off(r, c + CH)) = make_uint4(yo[0], yo[1], yo[2], yo[3]);
-                }
-            } else {
-#pragma unroll
-                for (int c = 0; c < 2 * CH; ++c) *reinterpret_cast<uint4*>(qs + swz_off(r, c)) = make_uint4(0, 0, 0, 0);
-            }
-            fence_proxy_async_smem();
-            mbar_arrive(&sh.q_full[k]);
+            uint8_t* qs = smem + Lay::Q0 + k * Lay::TILE;   // Q' tile; reused for the output tile
 
             // ---- main loop over key tiles
             const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
@@ -278,21 +314,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
                 for (int c = 0; c < 4; ++c) tmem_ld32(t_s + 32 * c, sr[c]);
                 tmem_wait_ld();
-                float mx = -INFINITY;
-                if (j == qtk) {   // diagonal tile: key column c sits at the same offset as query row r
+                const bool diag = (j == qtk);
+                if (diag) {   // diagonal tile: key column c sits at the same offset as query row r
 #pragma unroll
                     for (int c = 0; c < 4; ++c)
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) {
+                        for (int e = 0; e < 32; ++e)
                             if (32 * c + e > r) sr[c][e] = __float_as_uint(-INFINITY);
-                            mx = fmaxf(mx, __uint_as_float(sr[c][e]));
-                        }
-                } else {
-#pragma unroll
-                    for (int c = 0; c < 4; ++c)
-#pragma unroll
-                        for (int e = 0; e < 32; ++e) mx = fmaxf(mx, __uint_as_float(sr[c][e]));
                 }
+                float mxs[8];   // eight independent running maxima instead of one serial chain
+#pragma unroll
+                for (int e = 0; e < 8; ++e) mxs[e] = __uint_as_float(sr[0][e]);
+#pragma unroll
+                for (int i = 8; i < 128; ++i) mxs[i & 7] = fmaxf(mxs[i & 7], __uint_as_float(sr[i >> 5][i & 31]));
+                const float mx = fmaxf(fmaxf(fmaxf(mxs[0], mxs[1]), fmaxf(mxs[2], mxs[3])),
+                                       fmaxf(fmaxf(mxs[4], mxs[5]), fmaxf(mxs[6], mxs[7])));
                 const float m_new = fmaxf(m_run, mx * sl2);
                 if (j == 0) {
                     m_run = m_new;
@@ -313,21 +349,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     tmem_wait_st();
                 }
                 const float neg_m = -m_run;
-                float sum = 0.f;
-                // P chunk c (16 columns of bf16 pairs) overwrites S columns 16c.., already in registers.
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    uint32_t pk[16];
-#pragma unroll
-                    for (int e = 0; e < 32; e += 2) {
-                        const float p0 = ex2(fmaf(__uint_as_float(sr[c][e]), sl2, neg_m));
-                        const float p1 = ex2(fmaf(__uint_as_float(sr[c][e + 1]), sl2, neg_m));
-                        sum += p0 + p1;
-                        pk[e >> 1] = pack_bf16x2(p0, p1);
-                    }
-                    tmem_st16(t_s + 16 * c, pk);
-                }
-                l_run += sum;
+                if (diag) l_run += row_exp_store<false>(sr, sl2, neg_m, t_s);
+                else l_run += row_exp_store<true>(sr, sl2, neg_m, t_s);
                 tmem_wait_st();
                 tc_fence_before();
                 mbar_arrive(&sh.p_full[k]);
@@ -335,10 +358,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             // ---- epilogue: O / l -> bf16 -> out[b, row, head, :]
             if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&sh.o_full[k], (nk - 1) & 1, p.err, abort));
             if (ok) {
+                // Every MMA of this tile has completed, so its Q' tile is free: stage O / l there (same
+                // 128-byte-swizzled layout as the output tensor map's box) and store it with TMA.
                 tc_fence_after();
                 const float inv_l = 1.0f / l_run;
-                uint4* dst = reinterpret_cast<uint4*>(
-                    p.out + ((static_cast<int64_t>(b) * p.L + row) * p.h_q + headk) * D);
 #pragma unroll
                 for (int c = 0; c < D / 32; ++c) {
                     uint32_t o[32];
@@ -348,11 +371,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
                     for (int e = 0; e < 16; ++e)
                         w[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv_l, __uint_as_float(o[2 * e + 1]) * inv_l);
-                    if (row < p.L) {
 #pragma unroll
-                        for (int v4 = 0; v4 < 4; ++v4)
-                            dst[4 * c + v4] = make_uint4(w[4 * v4], w[4 * v4 + 1], w[4 * v4 + 2], w[4 * v4 + 3]);
-                    }
+                    for (int v4 = 0; v4 < 4; ++v4)
+                        *reinterpret_cast<uint4*>(qs + swz_off(r, 4 * c + v4)) =
+                            make_uint4(w[4 * v4], w[4 * v4 + 1], w[4 * v4 + 2], w[4 * v4 + 3]);
+                }
+                fence_proxy_async_smem();
+                named_barrier_sync(1 + k, 128);
+                if (r == 0) {   // rows >= L of the box are clipped by the store
+#pragma unroll
+                    for (int h = 0; h < D / 64; ++h) tma_store_4d(&tm_o, qs + h * Lay::SUB, h * 64, headk, qtk * BM, b);
+                    bulk_commit_group();
+                    bulk_wait_group_read0();
                 }
             }
         }
@@ -362,6 +392,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             const uint32_t tile_bytes = static_cast<uint32_t>(BN * D * 2);
             const int kv_plane = b * p.h_kv + u;
             int issued_k = 0, issued_v = 0;
+            // Q' tiles of the pair (query tile qt_k of head head_k), 128 rows from row qt_k * BM.
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                const int nk = k ? n1 : n0;
+                if (nk == 0) continue;
+                const int head = u * p.g + (k ? idx1 : idx0) % p.g;
+                mbar_arrive_expect_tx(&sh.q_full[k], static_cast<uint32_t>(BM * D * 2));
+                uint8_t* qdst = smem + Lay::Q0 + k * Lay::TILE;
+#pragma unroll
+                for (int h = 0; h < D / 64; ++h)
+                    tma_load_3d(qdst + h * Lay::SUB, &tm_q, &sh.q_full[k], h * 64, (nk - 1) * BM, b * p.h_q + head);
+            }
             for (int j = 0; j < nmax; ++j) {
                 const int ks = j % KSTAGES;
                 if (j >= KSTAGES && !mbar_wait(&sh.k_empty[ks], ((j / KSTAGES) - 1) & 1, p.err, abort)) break;
@@ -379,6 +421,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 issued_v = j + 1;
             }
             // Drain: never leave the CTA with copies still landing in its shared memory.
+            if (n0 > 0) mbar_wait(&sh.q_full[0], 0, p.err, nullptr);
+            if (n1 > 0) mbar_wait(&sh.q_full[1], 0, p.err, nullptr);
             for (int j = (issued_k > KSTAGES ? issued_k - KSTAGES : 0); j < issued_k; ++j)
                 mbar_wait(&sh.k_full[j % KSTAGES], (j / KSTAGES) & 1, p.err, nullptr);
             for (int j = (issued_v > VSTAGES ? issued_v - VSTAGES : 0); j < issued_v; ++j)
@@ -394,8 +438,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             const uint32_t v_addr0 = smem_u32(smem + Lay::V0);
             bool ok = nmax > 0;
             const int n[2] = {n0, n1};
-            for (int k = 0; k < 2 && ok; ++k)
-                if (n[k] > 0) ok = mbar_wait(&sh.q_full[k], 0, p.err, abort);
             // S_k = Q_k K_j^T : M=128 (query rows), N=128 (key rows), K=D in steps of 16.
             auto issue_s = [&](int k, int ks) {
                 const uint32_t qa = q_addr0 + k * Lay::TILE;
@@ -418,9 +460,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             };
             if (ok) ok = mbar_wait(&sh.k_full[0], 0, p.err, abort);
             if (ok) {
-                tc_fence_after();
-                for (int k = 0; k < 2; ++k)
+                // S_k of the first key tile as soon as query tile k is in shared memory.
+                for (int k = 0; k < 2 && ok; ++k)
                     if (n[k] > 0) {
+                        ok = mbar_wait(&sh.q_full[k], 0, p.err, abort);
+                        if (!ok) break;
+                        tc_fence_after();
                         issue_s(k, 0);
                         umma_commit(&sh.s_full[k]);
                     }

@@ -57,8 +57,8 @@ extern "C" {
  *   out [B, L, h_q,  d]   head_t rows, i.e. the concatenation [head_1 | ... | head_hq]
  * Positions are 0 .. L-1 in every batch row.  d in {64, 128}; h_q % h_kv == 0; any L >= 1
  * (a ragged last tile is handled).  B == 0 or L == 0 is a no-op that returns GQA_OK.
- * Uses an internal device workspace (rotated K and a cos/sin table, about
- * B*h_kv*L*d*2 + L*d*4 bytes), grown on demand and kept until gqa_release().
+ * Uses an internal device workspace (rotated Q and K, B*(h_q+h_kv)*L*d*2 bytes), grown on
+ * demand and kept until gqa_release().
  * theta is the RoPE base (Qwen2: 1e6).
  */
 GQA_API int gqa_prefill(const void* q, const void* k, const void* v, void* out,
