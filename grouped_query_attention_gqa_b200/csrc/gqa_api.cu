@@ -167,10 +167,11 @@ int launch_prefill(DeviceState* st, const void* q, const void* k, const void* v,
     const int prep_blocks = (L + PREP_POS - 1) / PREP_POS;
     prep_kernel<D><<<prep_blocks, PREP_THREADS, 0, g_stream>>>(static_cast<const __nv_bfloat16*>(q),
                                                                static_cast<const __nv_bfloat16*>(k), qr, kr, B, L,
-                                                               h_q, h_kv, static_cast<double>(theta));
+                                                               h_q, h_kv, std::log2(static_cast<double>(theta)));
     if (cudaGetLastError() != cudaSuccess) return GQA_ERR_LAUNCH;
 
     Params p;
+    p.out = static_cast<__nv_bfloat16*>(out);
     p.B = B;
     p.L = L;
     p.h_q = h_q;
@@ -180,9 +181,11 @@ int launch_prefill(DeviceState* st, const void* q, const void* k, const void* v,
     p.tiles_per_group = p.n_qtiles * p.g;
     p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
     p.err = st->err;
-    const int pairs = (p.tiles_per_group + 1) / 2;
-    const long long grid = static_cast<long long>(pairs) * B * h_kv;
-    if (grid > 0x7fffffffLL) return GQA_ERR_DIMS;
+    const long long total = static_cast<long long>((p.tiles_per_group + 1) / 2) * B * h_kv;
+    if (total > 0x7fffffffLL) return GQA_ERR_DIMS;
+    p.total_work = static_cast<int>(total);
+    // Persistent: one CTA per SM (each holds a whole SM's tensor memory), at most one per work item.
+    const int grid = static_cast<int>(total < st->num_sms ? total : st->num_sms);
     if (cudaFuncSetAttribute(attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, Layout<D>::DYN) !=
         cudaSuccess)
         return GQA_ERR_LAUNCH;
@@ -191,7 +194,7 @@ int launch_prefill(DeviceState* st, const void* q, const void* k, const void* v,
     if (cudaFuncGetAttributes(&fa, attn_kernel<D>) != cudaSuccess || fa.numRegs != LAUNCH_REGS)
         return GQA_ERR_LAUNCH;
     mark(g_ev_start);
-    attn_kernel<D><<<static_cast<unsigned>(grid), NUM_THREADS, Layout<D>::DYN, g_stream>>>(tm_q, tm_k, tm_v, tm_o, p);
+    attn_kernel<D><<<grid, NUM_THREADS, Layout<D>::DYN, g_stream>>>(tm_q, tm_k, tm_v, tm_o, p);
     if (cudaGetLastError() != cudaSuccess) return GQA_ERR_LAUNCH;
     mark(g_ev_stop);
     return GQA_OK;

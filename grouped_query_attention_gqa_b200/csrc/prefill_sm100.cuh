@@ -14,21 +14,24 @@
 //    streaming, bandwidth-bound pass; rotating there instead of in the attention kernel takes the
 //    rotation (and its latency) off the start of every attention CTA, and every K' tile is read by
 //    ~L/256 * g query tiles, so rotating K once beats rotating it on each use.
-//  * attn_kernel: one CTA per pair of 128-row query tiles of the same (b, KV group); Q', K' and V
-//    tiles arrive by TMA; each K'/V tile is brought into shared memory once and consumed by both
-//    query tiles (GQA reuse inside the CTA; the remaining heads of the group hit the same tiles in
-//    L2).  The output tile is staged in the (by then idle) Q' tile and written by a TMA store.
+//  * attn_kernel: persistent, one CTA per SM.  Each CTA walks a list of work items, each a pair of
+//    128-row query tiles of the same (b, KV group), heaviest first.  Q', K' and V tiles arrive by TMA;
+//    each K'/V tile is brought into shared memory once and consumed by both query tiles (GQA reuse
+//    inside the CTA; the remaining heads of the group hit the same tiles in L2).  Barrier phases run
+//    on across items, so the next pair's Q' is loaded as soon as the last S of the current pair has
+//    finished and its first S starts while the current pair's output is still being written.
 //
 // Warp roles (384 threads, three warpgroups):
 //   warps 0-3  softmax for query tile 0   (thread = query row = TMEM lane)
 //   warps 4-7  softmax for query tile 1
-//   warp  8    TMA producer (K', V tiles; 2-stage rings)
+//   warp  8    TMA producer of K', V tiles (2-stage rings)
 //   warp  9    tcgen05 MMA issuer (one thread); also owns the TMEM allocation
-//   warps 10-11 idle
+//   warp 10    TMA producer of the Q' tiles (one buffer per query tile)
+//   warp 11    idle
 // Each SM sub-partition hosts three warps, which caps a uniform budget at 168
-// registers; the third warpgroup hands 112 of its registers per thread to the
-// two softmax warpgroups (setmaxnreg), which then hold a full 128-column score
-// row in registers.
+// registers; the third warpgroup hands 88 of its registers per thread to the
+// two softmax warpgroups (setmaxnreg: 208 / 208 / 80), which then hold a full
+// 128-column score row in registers.
 // Tensor memory (512 columns): S0 [0,128) S1 [128,256) O0 [256,256+d) O1 [.., +d);
 // P_k (bf16, two per column) overwrites the first 64 columns of S_k.
 #pragma once
@@ -50,34 +53,43 @@ constexpr int KSTAGES = 2;
 constexpr int VSTAGES = 2;
 constexpr int NUM_WARPS = 12;
 constexpr int NUM_THREADS = NUM_WARPS * 32;
-constexpr int WARP_TMA = 8;
+constexpr int WARP_TMA = 8;     // K'/V producer
 constexpr int WARP_MMA = 9;
+constexpr int WARP_QLOAD = 10;  // Q' producer
 // Register split.  setmaxnreg.inc waits until the registers exist in the block's own
-// allocation (threads x launch registers), so the shares must add up to exactly that; the
-// host refuses to launch if ptxas gave the kernel any other count than LAUNCH_REGS.
+// allocation (threads x launch registers), so the shares must not add up to more than that;
+// the host refuses to launch if ptxas gave the kernel any other count than LAUNCH_REGS.
 constexpr int LAUNCH_REGS = 168;
-constexpr int SOFTMAX_REGS = 224;
-constexpr int OTHER_REGS = 56;
-static_assert(256 * SOFTMAX_REGS + 128 * OTHER_REGS == NUM_THREADS * LAUNCH_REGS, "register split");
+constexpr int SOFTMAX_REGS = 208;
+constexpr int OTHER_REGS = 80;
+static_assert(256 * SOFTMAX_REGS + 128 * OTHER_REGS <= NUM_THREADS * LAUNCH_REGS, "register split");
 constexpr uint32_t TMEM_COLS = 512;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: O is rescaled only when the max grows by > 2^8
 // Of every 8 consecutive exponentials of a row (off the diagonal tile), this many run on the FMA
 // pipe (exp2_poly) and the rest on the ex2 unit.
 #ifndef GQA_EXP_POLY_OF_8
-#define GQA_EXP_POLY_OF_8 0
+#define GQA_EXP_POLY_OF_8 1
 #endif
 // 1: round P to bf16 with integer ops instead of the conversion instruction.
 #ifndef GQA_PACK_INT
 #define GQA_PACK_INT 0
 #endif
+// 1: the output tile is staged in the pair's Q' tile and written by a TMA store (the tile is handed
+// back to the producer after the store has read it); 0: every thread stores its row directly and
+// the Q' tile is handed back as soon as the pair's last S has finished.
+#ifndef GQA_EPILOGUE_TMA
+#define GQA_EPILOGUE_TMA 1
+#endif
 constexpr int PREP_POS = 8;                 // positions per CTA of the prep kernel
-constexpr int PREP_UNROLL = 4;              // work items per thread in flight
+constexpr int PREP_UNROLL = 8;              // work items per thread in flight
 constexpr int PREP_THREADS = 256;
 
 struct Params {
+    __nv_bfloat16* out;        // [B, L, h_q, D]
     int B, L, h_q, h_kv, g;
     int n_qtiles;              // ceil(L / BM)
     int tiles_per_group;       // n_qtiles * g
+    int total_work;            // tile pairs in all: ceil(tiles_per_group / 2) * B * h_kv
     float scale_log2;          // log2(e) / sqrt(D)
     int* err;
 };
@@ -95,7 +107,7 @@ struct Layout {
 };
 
 struct alignas(8) Shared {
-    uint64_t q_full[2];
+    uint64_t q_full[2], q_empty[2];
     uint64_t k_full[KSTAGES], k_empty[KSTAGES];
     uint64_t v_full[VSTAGES], v_empty[VSTAGES];
     uint64_t s_full[2], p_full[2], o_full[2];
@@ -108,11 +120,11 @@ struct alignas(8) Shared {
 // prep_kernel: for positions [p0, p0+PREP_POS): the cos/sin table, then every Q and K row at those
 // positions rotated into Q' [B*h_q, L, D] and K' [B*h_kv, L, D].
 template <int D>
-__global__ void __launch_bounds__(PREP_THREADS) prep_kernel(const __nv_bfloat16* __restrict__ q,
+__global__ void __launch_bounds__(PREP_THREADS, 2) prep_kernel(const __nv_bfloat16* __restrict__ q,
                                                             const __nv_bfloat16* __restrict__ k,
                                                             __nv_bfloat16* __restrict__ qr,
                                                             __nv_bfloat16* __restrict__ kr, int B, int L,
-                                                            int h_q, int h_kv, double theta) {
+                                                            int h_q, int h_kv, double log2_theta) {
     constexpr int H = D / 2;
     constexpr int CH = D / 16;   // one work item = 8 pairs: a 16-byte chunk of the first half + its partner
     __shared__ float2 tab[PREP_POS][H];
@@ -152,7 +164,8 @@ __global__ void __launch_bounds__(PREP_THREADS) prep_kernel(const __nv_bfloat16*
     int base = threadIdx.x;
     load_round(base);
 
-    for (int i = threadIdx.x; i < H; i += blockDim.x) finv[i] = rope_inv_freq(i, D, theta);
+    // theta^(-2i/D) = 2^(-(2i/D) * log2(theta))
+    for (int i = threadIdx.x; i < H; i += blockDim.x) finv[i] = exp2(-(2.0 * i / D) * log2_theta);
     __syncthreads();
     for (int e = threadIdx.x; e < PREP_POS * H; e += blockDim.x) {
         const int pp = e / H, i = e % H;
@@ -224,6 +237,32 @@ __device__ __forceinline__ uint32_t swz_off(int r, int cc) {
     return static_cast<uint32_t>((cc >> 3) * (BM * 128) + r * 128 + (((cc & 7) ^ (r & 7)) << 4));
 }
 
+// One work item = a pair of 128-row query tiles of one (b, KV group).  Items are numbered heaviest
+// first: item w = pair * (B * h_kv) + (b * h_kv + u), and pair q holds tiles 2q and 2q+1 of the group's
+// list (query tile descending, head ascending), so both tiles of a pair need about the same number of
+// key tiles.
+struct PairWork {
+    int b, u, n0, n1, head0, head1;
+};
+
+__device__ __forceinline__ PairWork pair_work(const Params& p, int w) {
+    PairWork r;
+    const int BH = p.B * p.h_kv;
+    const int pair = w / BH, bu = w % BH;
+    r.b = bu / p.h_kv;
+    r.u = bu % p.h_kv;
+    const int i0 = 2 * pair, i1 = 2 * pair + 1;
+    r.n0 = i0 < p.tiles_per_group ? p.n_qtiles - i0 / p.g : 0;   // tile needs key tiles 0 .. qt (BM == BN)
+    r.n1 = i1 < p.tiles_per_group ? p.n_qtiles - i1 / p.g : 0;
+    r.head0 = r.u * p.g + i0 % p.g;
+    r.head1 = r.u * p.g + i1 % p.g;
+    return r;
+}
+
+// The r-th item of persistent CTA c out of G: rounds of G consecutive items, every other round
+// reversed (snake order), so the heaviest-first list spreads evenly over the CTAs.
+__device__ __forceinline__ int work_item(int r, int c, int G) { return r * G + ((r & 1) ? (G - 1 - c) : c); }
+
 template <int D>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -236,22 +275,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-
-    // ---- work assignment: blockIdx -> (pair, b, u); pairs of the heaviest query tiles come first.
-    const int BH = p.B * p.h_kv;
-    const int pair = blockIdx.x / BH;
-    const int bu = blockIdx.x % BH;
-    const int b = bu / p.h_kv;
-    const int u = bu % p.h_kv;
-    // Tile k of the pair: query tile qt_k of head head_k; it needs key tiles 0 .. qt_k (BM == BN).
-    const int idx0 = 2 * pair, idx1 = 2 * pair + 1;
-    const int n0 = idx0 < p.tiles_per_group ? p.n_qtiles - idx0 / p.g : 0;
-    const int n1 = idx1 < p.tiles_per_group ? p.n_qtiles - idx1 / p.g : 0;
-    const int nmax = n0 > n1 ? n0 : n1;
+    const int G = gridDim.x, cta = blockIdx.x;
 
     if (threadIdx.x == 0) {
-        mbar_init(&sh.q_full[0], 1);
-        mbar_init(&sh.q_full[1], 1);
+        for (int k = 0; k < 2; ++k) {
+            mbar_init(&sh.q_full[k], 1);
+            mbar_init(&sh.q_empty[k], 1);
+            mbar_init(&sh.s_full[k], 1);
+            mbar_init(&sh.p_full[k], 128);
+            mbar_init(&sh.o_full[k], 1);
+        }
         for (int s = 0; s < KSTAGES; ++s) {
             mbar_init(&sh.k_full[s], 1);
             mbar_init(&sh.k_empty[s], 1);
@@ -259,11 +292,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int s = 0; s < VSTAGES; ++s) {
             mbar_init(&sh.v_full[s], 1);
             mbar_init(&sh.v_empty[s], 1);
-        }
-        for (int k = 0; k < 2; ++k) {
-            mbar_init(&sh.s_full[k], 1);
-            mbar_init(&sh.p_full[k], 128);
-            mbar_init(&sh.o_full[k], 1);
         }
         mbar_init(&sh.mma_done, 1);
         sh.abort = 0;
@@ -273,8 +301,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tmem_alloc(&sh.tmem_base, TMEM_COLS);
         tmem_relinquish();
     }
+    if (warp == WARP_QLOAD && lane == 0) prefetch_tensormap(&tm_q);
     if (warp == WARP_TMA && lane == 0) {
-        prefetch_tensormap(&tm_q);
         prefetch_tensormap(&tm_k);
         prefetch_tensormap(&tm_v);
         prefetch_tensormap(&tm_o);
@@ -289,26 +317,29 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     else regs_decrease<OTHER_REGS>();
 
     if (warp < 8) {
-        // ================================================================ softmax / epilogue
+        // ================================================================ softmax / epilogue of tile k
         const int k = warp >> 2;
         const int r = (warp & 3) * 32 + lane;   // query row in the tile == TMEM lane
-        const int idx = k ? idx1 : idx0;
-        const int nk = k ? n1 : n0;
-        const int qtk = nk - 1;
-        const int headk = u * p.g + idx % p.g;
-        if (nk > 0) {
-            uint8_t* qs = smem + Lay::Q0 + k * Lay::TILE;   // Q' tile; reused for the output tile
-
-            // ---- main loop over key tiles
-            const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-            const uint32_t t_s = tmem + lane_base + static_cast<uint32_t>(k * 128);
-            const uint32_t t_o = tmem + lane_base + static_cast<uint32_t>(256 + k * D);
-            const float sl2 = p.scale_log2;
+        const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+        const uint32_t t_s = tmem + lane_base + static_cast<uint32_t>(k * 128);
+        const uint32_t t_o = tmem + lane_base + static_cast<uint32_t>(256 + k * D);
+        const float sl2 = p.scale_log2;
+        uint32_t s_seen = 0;   // S_k results consumed (s_full phases)
+        uint32_t o_seen = 0;   // PV_k products issued for the pairs handled so far (o_full phases)
+        bool ok = true;
+        for (int it = 0; ok; ++it) {
+            const int w = work_item(it, cta, G);
+            if (w >= p.total_work) break;
+            const PairWork pw = pair_work(p, w);
+            const int nk = k ? pw.n1 : pw.n0;
+            if (nk == 0) continue;
+            const int qtk = nk - 1;
+            const int headk = k ? pw.head1 : pw.head0;
             float m_run = -INFINITY, l_run = 0.f;
-            bool ok = true;
             for (int j = 0; j < nk; ++j) {
-                ok = __all_sync(0xffffffffu, mbar_wait(&sh.s_full[k], j & 1, p.err, abort));
+                ok = __all_sync(0xffffffffu, mbar_wait(&sh.s_full[k], s_seen & 1, p.err, abort));
                 if (!ok) break;
+                ++s_seen;
                 tc_fence_after();
                 uint32_t sr[4][32];
 #pragma unroll
@@ -355,78 +386,137 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 tc_fence_before();
                 mbar_arrive(&sh.p_full[k]);
             }
-            // ---- epilogue: O / l -> bf16 -> out[b, row, head, :]
-            if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&sh.o_full[k], (nk - 1) & 1, p.err, abort));
-            if (ok) {
-                // Every MMA of this tile has completed, so its Q' tile is free: stage O / l there (same
-                // 128-byte-swizzled layout as the output tensor map's box) and store it with TMA.
-                tc_fence_after();
-                const float inv_l = 1.0f / l_run;
+            if (!ok) break;
+            // ---- epilogue: O / l -> bf16 -> out[b, row, head, :].  The next pair's S_k may already be
+            // running; its first PV_k (which overwrites O_k) waits for this warpgroup's next P.
+            o_seen += nk;
+            ok = __all_sync(0xffffffffu, mbar_wait(&sh.o_full[k], (o_seen - 1) & 1, p.err, abort));
+            if (!ok) break;
+            tc_fence_after();
+            const float inv_l = 1.0f / l_run;
+#if GQA_EPILOGUE_TMA
+            // Every MMA reading this pair's Q' tile has finished: stage O / l there (the 128-byte
+            // swizzled layout of the output tensor map's box), store it with TMA, then hand the tile
+            // back to the producer for the next pair.
+            uint8_t* qs = smem + Lay::Q0 + k * Lay::TILE;
 #pragma unroll
-                for (int c = 0; c < D / 32; ++c) {
-                    uint32_t o[32];
-                    tmem_ld32(t_o + 32 * c, o);
-                    tmem_wait_ld();
-                    uint32_t w[16];
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t o[32];
+                tmem_ld32(t_o + 32 * c, o);
+                tmem_wait_ld();
+                uint32_t wv[16];
 #pragma unroll
-                    for (int e = 0; e < 16; ++e)
-                        w[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv_l, __uint_as_float(o[2 * e + 1]) * inv_l);
+                for (int e = 0; e < 16; ++e)
+                    wv[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv_l, __uint_as_float(o[2 * e + 1]) * inv_l);
+#pragma unroll
+                for (int v4 = 0; v4 < 4; ++v4)
+                    *reinterpret_cast<uint4*>(qs + swz_off(r, 4 * c + v4)) =
+                        make_uint4(wv[4 * v4], wv[4 * v4 + 1], wv[4 * v4 + 2], wv[4 * v4 + 3]);
+            }
+            tc_fence_before();
+            fence_proxy_async_smem();
+            named_barrier_sync(1 + k, 128);
+            if (r == 0) {   // rows >= L of the box are clipped by the store
+#pragma unroll
+                for (int h = 0; h < D / 64; ++h) tma_store_4d(&tm_o, qs + h * Lay::SUB, h * 64, headk, qtk * BM, pw.b);
+                bulk_commit_group();
+                bulk_wait_group_read0();
+                mbar_arrive(&sh.q_empty[k]);
+            }
+#else
+            const int row = qtk * BM + r;
+            uint4* dst = reinterpret_cast<uint4*>(
+                p.out + ((static_cast<int64_t>(pw.b) * p.L + row) * p.h_q + headk) * D);
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t o[32];
+                tmem_ld32(t_o + 32 * c, o);
+                tmem_wait_ld();
+                uint32_t wv[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e)
+                    wv[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv_l, __uint_as_float(o[2 * e + 1]) * inv_l);
+                if (row < p.L) {
 #pragma unroll
                     for (int v4 = 0; v4 < 4; ++v4)
-                        *reinterpret_cast<uint4*>(qs + swz_off(r, 4 * c + v4)) =
-                            make_uint4(w[4 * v4], w[4 * v4 + 1], w[4 * v4 + 2], w[4 * v4 + 3]);
-                }
-                fence_proxy_async_smem();
-                named_barrier_sync(1 + k, 128);
-                if (r == 0) {   // rows >= L of the box are clipped by the store
-#pragma unroll
-                    for (int h = 0; h < D / 64; ++h) tma_store_4d(&tm_o, qs + h * Lay::SUB, h * 64, headk, qtk * BM, b);
-                    bulk_commit_group();
-                    bulk_wait_group_read0();
+                        dst[4 * c + v4] = make_uint4(wv[4 * v4], wv[4 * v4 + 1], wv[4 * v4 + 2], wv[4 * v4 + 3]);
                 }
             }
+            tc_fence_before();
+#endif
         }
     } else if (warp == WARP_TMA) {
         // ================================================================ TMA producer
-        if (lane == 0 && nmax > 0) {
+        if (lane == 0) {
             const uint32_t tile_bytes = static_cast<uint32_t>(BN * D * 2);
-            const int kv_plane = b * p.h_kv + u;
-            int issued_k = 0, issued_v = 0;
-            // Q' tiles of the pair (query tile qt_k of head head_k), 128 rows from row qt_k * BM.
+            uint32_t kv = 0;                 // K/V tiles issued so far (ring position)
+            bool ok = true;
+            for (int it = 0; ok; ++it) {
+                const int w = work_item(it, cta, G);
+                if (w >= p.total_work) break;
+                const PairWork pw = pair_work(p, w);
+                const int n[2] = {pw.n0, pw.n1};
+                const int nmax = n[0] > n[1] ? n[0] : n[1];
+                const int kv_plane = pw.b * p.h_kv + pw.u;
+                for (int j = 0; j < nmax && ok; ++j, ++kv) {
+                    const int ks = kv % KSTAGES;
+                    if (kv >= KSTAGES && !mbar_wait(&sh.k_empty[ks], ((kv / KSTAGES) - 1) & 1, p.err, abort)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&sh.k_full[ks], tile_bytes);
+                    uint8_t* kdst = smem + Lay::K0 + ks * Lay::TILE;
 #pragma unroll
-            for (int k = 0; k < 2; ++k) {
-                const int nk = k ? n1 : n0;
-                if (nk == 0) continue;
-                const int head = u * p.g + (k ? idx1 : idx0) % p.g;
-                mbar_arrive_expect_tx(&sh.q_full[k], static_cast<uint32_t>(BM * D * 2));
-                uint8_t* qdst = smem + Lay::Q0 + k * Lay::TILE;
+                    for (int h = 0; h < D / 64; ++h)
+                        tma_load_3d(kdst + h * Lay::SUB, &tm_k, &sh.k_full[ks], h * 64, j * BN, kv_plane);
+                    const int vs = kv % VSTAGES;
+                    if (kv >= VSTAGES && !mbar_wait(&sh.v_empty[vs], ((kv / VSTAGES) - 1) & 1, p.err, abort)) {
+                        // K tile kv was issued without its V: count it so the drain below waits for it.
+                        ++kv;
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&sh.v_full[vs], tile_bytes);
+                    uint8_t* vdst = smem + Lay::V0 + vs * Lay::TILE;
 #pragma unroll
-                for (int h = 0; h < D / 64; ++h)
-                    tma_load_3d(qdst + h * Lay::SUB, &tm_q, &sh.q_full[k], h * 64, (nk - 1) * BM, b * p.h_q + head);
-            }
-            for (int j = 0; j < nmax; ++j) {
-                const int ks = j % KSTAGES;
-                if (j >= KSTAGES && !mbar_wait(&sh.k_empty[ks], ((j / KSTAGES) - 1) & 1, p.err, abort)) break;
-                mbar_arrive_expect_tx(&sh.k_full[ks], tile_bytes);
-                uint8_t* kdst = smem + Lay::K0 + ks * Lay::TILE;
-#pragma unroll
-                for (int h = 0; h < D / 64; ++h) tma_load_3d(kdst + h * Lay::SUB, &tm_k, &sh.k_full[ks], h * 64, j * BN, kv_plane);
-                issued_k = j + 1;
-                const int vs = j % VSTAGES;
-                if (j >= VSTAGES && !mbar_wait(&sh.v_empty[vs], ((j / VSTAGES) - 1) & 1, p.err, abort)) break;
-                mbar_arrive_expect_tx(&sh.v_full[vs], tile_bytes);
-                uint8_t* vdst = smem + Lay::V0 + vs * Lay::TILE;
-#pragma unroll
-                for (int h = 0; h < D / 64; ++h) tma_load_4d(vdst + h * Lay::SUB, &tm_v, &sh.v_full[vs], h * 64, u, j * BN, b);
-                issued_v = j + 1;
+                    for (int h = 0; h < D / 64; ++h)
+                        tma_load_4d(vdst + h * Lay::SUB, &tm_v, &sh.v_full[vs], h * 64, pw.u, j * BN, pw.b);
+                }
             }
             // Drain: never leave the CTA with copies still landing in its shared memory.
-            if (n0 > 0) mbar_wait(&sh.q_full[0], 0, p.err, nullptr);
-            if (n1 > 0) mbar_wait(&sh.q_full[1], 0, p.err, nullptr);
-            for (int j = (issued_k > KSTAGES ? issued_k - KSTAGES : 0); j < issued_k; ++j)
+            for (uint32_t j = (kv > KSTAGES ? kv - KSTAGES : 0); j < kv; ++j)
                 mbar_wait(&sh.k_full[j % KSTAGES], (j / KSTAGES) & 1, p.err, nullptr);
-            for (int j = (issued_v > VSTAGES ? issued_v - VSTAGES : 0); j < issued_v; ++j)
+            for (uint32_t j = (kv > VSTAGES ? kv - VSTAGES : 0); j < kv; ++j)
                 mbar_wait(&sh.v_full[j % VSTAGES], (j / VSTAGES) & 1, p.err, nullptr);
+        }
+    } else if (warp == WARP_QLOAD) {
+        // ================================================================ Q' producer
+        if (lane == 0) {
+            uint32_t qn[2] = {0u, 0u};   // Q' tiles issued into buffer k so far
+            bool ok = true;
+            for (int it = 0; ok; ++it) {
+                const int w = work_item(it, cta, G);
+                if (w >= p.total_work) break;
+                const PairWork pw = pair_work(p, w);
+                for (int k = 0; k < 2 && ok; ++k) {
+                    const int nk = k ? pw.n1 : pw.n0;
+                    if (nk == 0) continue;
+                    // Wait until the buffer has been handed back (see GQA_EPILOGUE_TMA).
+                    if (qn[k] > 0 && !mbar_wait(&sh.q_empty[k], (qn[k] - 1) & 1, p.err, abort)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&sh.q_full[k], static_cast<uint32_t>(BM * D * 2));
+                    uint8_t* qdst = smem + Lay::Q0 + k * Lay::TILE;
+                    const int head = k ? pw.head1 : pw.head0;
+#pragma unroll
+                    for (int h = 0; h < D / 64; ++h)
+                        tma_load_3d(qdst + h * Lay::SUB, &tm_q, &sh.q_full[k], h * 64, (nk - 1) * BM, pw.b * p.h_q + head);
+                    ++qn[k];
+                }
+            }
+            for (int k = 0; k < 2; ++k)   // drain
+                if (qn[k] > 0) mbar_wait(&sh.q_full[k], (qn[k] - 1) & 1, p.err, nullptr);
         }
     } else if (warp == WARP_MMA) {
         // ================================================================ MMA issuer
@@ -436,8 +526,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             const uint32_t q_addr0 = smem_u32(smem + Lay::Q0);
             const uint32_t k_addr0 = smem_u32(smem + Lay::K0);
             const uint32_t v_addr0 = smem_u32(smem + Lay::V0);
-            bool ok = nmax > 0;
-            const int n[2] = {n0, n1};
             // S_k = Q_k K_j^T : M=128 (query rows), N=128 (key rows), K=D in steps of 16.
             auto issue_s = [&](int k, int ks) {
                 const uint32_t qa = q_addr0 + k * Lay::TILE;
@@ -458,45 +546,62 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                             sw128_desc(va + kk * 16 * 128, Lay::SUB, 1024), IDESC_PV, (acc || kk > 0) ? 1u : 0u);
                 }
             };
-            if (ok) ok = mbar_wait(&sh.k_full[0], 0, p.err, abort);
-            if (ok) {
+            uint32_t kv = 0;               // K/V tiles consumed (ring position)
+            uint32_t qn[2] = {0u, 0u};     // q_full phases consumed per buffer
+            uint32_t pn[2] = {0u, 0u};     // p_full phases consumed per tile
+            bool ok = true;
+            for (int it = 0; ok; ++it) {
+                const int w = work_item(it, cta, G);
+                if (w >= p.total_work) break;
+                const PairWork pw = pair_work(p, w);
+                const int n[2] = {pw.n0, pw.n1};
+                const int nmax = n[0] > n[1] ? n[0] : n[1];
                 // S_k of the first key tile as soon as query tile k is in shared memory.
-                for (int k = 0; k < 2 && ok; ++k)
-                    if (n[k] > 0) {
-                        ok = mbar_wait(&sh.q_full[k], 0, p.err, abort);
-                        if (!ok) break;
-                        tc_fence_after();
-                        issue_s(k, 0);
-                        umma_commit(&sh.s_full[k]);
-                    }
-                umma_commit(&sh.k_empty[0]);
+                const int ks0 = kv % KSTAGES;
+                ok = mbar_wait(&sh.k_full[ks0], (kv / KSTAGES) & 1, p.err, abort);
+                for (int k = 0; k < 2 && ok; ++k) {
+                    if (n[k] == 0) continue;
+                    ok = mbar_wait(&sh.q_full[k], qn[k] & 1, p.err, abort);
+                    if (!ok) break;
+                    ++qn[k];
+                    tc_fence_after();
+                    issue_s(k, ks0);
+                    umma_commit(&sh.s_full[k]);
+                    if (!GQA_EPILOGUE_TMA && n[k] == 1) umma_commit(&sh.q_empty[k]);   // last S on buffer k
+                }
+                if (!ok) break;
+                umma_commit(&sh.k_empty[ks0]);
                 for (int j = 0; j < nmax && ok; ++j) {
-                    const int vs = j % VSTAGES;
-                    ok = mbar_wait(&sh.v_full[vs], (j / VSTAGES) & 1, p.err, abort);
+                    const uint32_t vi = kv + j;
+                    const int vs = vi % VSTAGES;
+                    ok = mbar_wait(&sh.v_full[vs], (vi / VSTAGES) & 1, p.err, abort);
                     if (!ok) break;
                     bool k_next = false;
+                    const uint32_t ki = kv + j + 1;
                     for (int k = 0; k < 2 && ok; ++k) {
                         if (j >= n[k]) continue;
-                        ok = mbar_wait(&sh.p_full[k], j & 1, p.err, abort);
+                        ok = mbar_wait(&sh.p_full[k], pn[k] & 1, p.err, abort);
                         if (!ok) break;
+                        ++pn[k];
                         tc_fence_after();
                         issue_pv(k, vs, j > 0);
                         umma_commit(&sh.o_full[k]);
                         if (j + 1 < n[k]) {
-                            const int ks = (j + 1) % KSTAGES;
                             if (!k_next) {
-                                ok = mbar_wait(&sh.k_full[ks], ((j + 1) / KSTAGES) & 1, p.err, abort);
+                                ok = mbar_wait(&sh.k_full[ki % KSTAGES], (ki / KSTAGES) & 1, p.err, abort);
                                 if (!ok) break;
                                 tc_fence_after();
                                 k_next = true;
                             }
-                            issue_s(k, ks);
+                            issue_s(k, ki % KSTAGES);
                             umma_commit(&sh.s_full[k]);
+                            if (!GQA_EPILOGUE_TMA && j + 2 == n[k]) umma_commit(&sh.q_empty[k]);
                         }
                     }
                     umma_commit(&sh.v_empty[vs]);
-                    if (k_next) umma_commit(&sh.k_empty[(j + 1) % KSTAGES]);
+                    if (k_next) umma_commit(&sh.k_empty[ki % KSTAGES]);
                 }
+                kv += nmax;
             }
             // Every MMA must have finished before the tensor memory is released.
             umma_commit(&sh.mma_done);
