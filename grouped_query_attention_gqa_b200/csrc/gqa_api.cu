@@ -133,6 +133,13 @@ int launch_prefill(DeviceState* st, const void* q, const void* k, const void* v,
     auto* qr = static_cast<__nv_bfloat16*>(st->ws);
     auto* kr = reinterpret_cast<__nv_bfloat16*>(static_cast<uint8_t*>(st->ws) + qr_bytes);
 
+    const int prep_blocks = (L + PREP_POS - 1) / PREP_POS;
+    prep_kernel<D><<<prep_blocks, PREP_THREADS, 0, g_stream>>>(static_cast<const __nv_bfloat16*>(q),
+                                                               static_cast<const __nv_bfloat16*>(k), qr, kr, B, L,
+                                                               h_q, h_kv, std::log2(static_cast<double>(theta)));
+    if (cudaGetLastError() != cudaSuccess) return GQA_ERR_LAUNCH;
+    // (the host work below overlaps the prep kernel)
+
     if (!get_encoder()) return GQA_ERR_LAUNCH;
     CUtensorMap tm_q, tm_k, tm_v, tm_o;
     const cuuint32_t box3[3] = {64, BM, 1};
@@ -161,14 +168,9 @@ int launch_prefill(DeviceState* st, const void* q, const void* k, const void* v,
                                     static_cast<cuuint64_t>(L), static_cast<cuuint64_t>(B)};
         const cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(h_q) * D * 2,
                                        static_cast<cuuint64_t>(L) * h_q * D * 2};
-        if (!encode_bf16(&tm_o, out, 4, dims, strides, box4)) return GQA_ERR_LAUNCH;
+        const cuuint32_t box_o[4] = {64, 1, 32, 1};   // one softmax warp's 32 rows, 64 columns
+        if (!encode_bf16(&tm_o, out, 4, dims, strides, box_o)) return GQA_ERR_LAUNCH;
     }
-
-    const int prep_blocks = (L + PREP_POS - 1) / PREP_POS;
-    prep_kernel<D><<<prep_blocks, PREP_THREADS, 0, g_stream>>>(static_cast<const __nv_bfloat16*>(q),
-                                                               static_cast<const __nv_bfloat16*>(k), qr, kr, B, L,
-                                                               h_q, h_kv, std::log2(static_cast<double>(theta)));
-    if (cudaGetLastError() != cudaSuccess) return GQA_ERR_LAUNCH;
 
     Params p;
     p.out = static_cast<__nv_bfloat16*>(out);

@@ -74,9 +74,14 @@ constexpr float kRescaleThreshold = 8.0f;   // log2 units: O is rescaled only wh
 #ifndef GQA_PACK_INT
 #define GQA_PACK_INT 0
 #endif
-// 1: the output tile is staged in the pair's Q' tile and written by a TMA store (the tile is handed
-// back to the producer after the store has read it); 0: every thread stores its row directly and
-// the Q' tile is handed back as soon as the pair's last S has finished.
+// 1: P is truncated to bf16 (one byte permute per pair, off the conversion unit) and the row sum l
+// accumulates the same truncated values, so the normalisation matches the weights the MMA uses.
+#ifndef GQA_PACK_TRUNC
+#define GQA_PACK_TRUNC 0
+#endif
+// Epilogue: each softmax warp stages its 32 output rows, one 64-column half at a time, in a 4 KB
+// slot of its own and writes them with TMA stores, so the Q' tile is handed back to the producer as
+// soon as the pair's last S has finished (GQA_EPILOGUE_TMA 1).  0: every thread stores its row directly.
 #ifndef GQA_EPILOGUE_TMA
 #define GQA_EPILOGUE_TMA 1
 #endif
@@ -101,7 +106,9 @@ struct Layout {
     static constexpr int Q0 = 0;
     static constexpr int K0 = 2 * TILE;
     static constexpr int V0 = K0 + KSTAGES * TILE;
-    static constexpr int BYTES = V0 + VSTAGES * TILE;
+    static constexpr int OSTAGE = 32 * 128;            // one warp's 32 rows x 64 columns, swizzled
+    static constexpr int O0 = V0 + VSTAGES * TILE;     // 8 softmax warps x OSTAGE
+    static constexpr int BYTES = O0 + 8 * OSTAGE;
     // At least 120 KB so that two CTAs never share an SM: each holds all 512 TMEM columns.
     static constexpr int DYN = (BYTES < 120 * 1024 ? 120 * 1024 : BYTES) + 1024;
 };
@@ -127,11 +134,15 @@ __global__ void __launch_bounds__(PREP_THREADS, 2) prep_kernel(const __nv_bfloat
                                                             int h_q, int h_kv, double log2_theta) {
     constexpr int H = D / 2;
     constexpr int CH = D / 16;   // one work item = 8 pairs: a 16-byte chunk of the first half + its partner
-    __shared__ float2 tab[PREP_POS][H];
+    // Table row pp holds the D/2 (cos, sin) pairs of position p0 + pp, one padding slot after every 8, so
+    // the 8 chunks of a row (read by 8 neighbouring lanes) fall in 8 different shared-memory banks.
+    constexpr int TROW = H + H / 8;
+    __shared__ float2 tab[PREP_POS * TROW];
     __shared__ double finv[H];
     const int p0 = blockIdx.x * PREP_POS;
     const int heads = h_q + h_kv;
-    const int items = B * heads * PREP_POS * CH;   // < 2^31: B * (h_q + h_kv) is checked on the host
+    const int bh_n = B * heads;
+    const int items = bh_n * PREP_POS * CH;   // < 2^31: B * (h_q + h_kv) is checked on the host
 
     // PREP_UNROLL items per thread per round, loads first, so each thread keeps several 32-byte reads in
     // flight (the pass is bandwidth bound); the first round's loads are issued before the table is built.
@@ -142,10 +153,12 @@ __global__ void __launch_bounds__(PREP_THREADS, 2) prep_kernel(const __nv_bfloat
 #pragma unroll
         for (int uidx = 0; uidx < PREP_UNROLL; ++uidx) {
             const int e = base + uidx * static_cast<int>(blockDim.x);
+            // item e: chunk fastest, then the row (b, head), then the position, so a warp works on 4 rows
+            // of one position and its table reads are 8 distinct addresses, each broadcast to 4 lanes.
             dst[uidx] = nullptr;
             cc[uidx] = e % CH;
-            ppp[uidx] = (e / CH) % PREP_POS;
-            const int bh = e / (CH * PREP_POS);
+            const int bh = (e / CH) % bh_n;
+            ppp[uidx] = e / (CH * bh_n);
             const int pos = p0 + ppp[uidx];
             if (e >= items || pos >= L) continue;
             const int b = bh / heads, h = bh % heads;
@@ -171,7 +184,7 @@ __global__ void __launch_bounds__(PREP_THREADS, 2) prep_kernel(const __nv_bfloat
         const int pp = e / H, i = e % H;
         float c = 1.f, s = 0.f;
         if (p0 + pp < L) rope_cossin(static_cast<double>(p0 + pp), finv[i], c, s);
-        tab[pp][i] = make_float2(c, s);
+        tab[pp * TROW + i + i / 8] = make_float2(c, s);
     }
     __syncthreads();
 
@@ -186,8 +199,8 @@ __global__ void __launch_bounds__(PREP_THREADS, 2) prep_kernel(const __nv_bfloat
             uint32_t xo[4], yo[4];
 #pragma unroll
             for (int w = 0; w < 4; ++w) {
-                const float2 c0 = tab[pp][8 * c + 2 * w];
-                const float2 c1 = tab[pp][8 * c + 2 * w + 1];
+                const float2 c0 = tab[pp * TROW + 9 * c + 2 * w];       // i = 8c + 2w, padded
+                const float2 c1 = tab[pp * TROW + 9 * c + 2 * w + 1];
                 float a0, b0, a1, b1;
                 rope_rotate(bf16lo_to_f32(xs[w]), bf16lo_to_f32(ys[w]), c0.x, c0.y, a0, b0);
                 rope_rotate(bf16hi_to_f32(xs[w]), bf16hi_to_f32(ys[w]), c1.x, c1.y, a1, b1);
@@ -224,8 +237,14 @@ __device__ __forceinline__ float row_exp_store(const uint32_t (&sr)[4][32], floa
             const float x1 = fmaf(__uint_as_float(sr[c][e + 1]), sl2, neg_m);
             const float p0 = (POLY && (e & 7) < GQA_EXP_POLY_OF_8) ? exp2_poly(x0) : ex2(x0);
             const float p1 = (POLY && ((e + 1) & 7) < GQA_EXP_POLY_OF_8) ? exp2_poly(x1) : ex2(x1);
+#if GQA_PACK_TRUNC
+            const uint32_t b0 = __float_as_uint(p0), b1 = __float_as_uint(p1);
+            pk[e >> 1] = __byte_perm(b0, b1, 0x7632);
+            acc[(e >> 1) & 3] += __uint_as_float(b0 & 0xFFFF0000u) + __uint_as_float(b1 & 0xFFFF0000u);
+#else
             acc[(e >> 1) & 3] += p0 + p1;
             pk[e >> 1] = pack_p(p0, p1);
+#endif
         }
         tmem_st16(t_s + 16 * c, pk);
     }
@@ -395,34 +414,38 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             tc_fence_after();
             const float inv_l = 1.0f / l_run;
 #if GQA_EPILOGUE_TMA
-            // Every MMA reading this pair's Q' tile has finished: stage O / l there (the 128-byte
-            // swizzled layout of the output tensor map's box), store it with TMA, then hand the tile
-            // back to the producer for the next pair.
-            uint8_t* qs = smem + Lay::Q0 + k * Lay::TILE;
+            // Rows 32*(warp&3) .. +31 of the tile, one 64-column half per pass: stage in this warp's slot
+            // (same 128-byte-swizzled layout as the output tensor map's 64 x 32 box), TMA-store, and wait
+            // for the store to have read the slot before the next pass.  Rows >= L are clipped.
+            uint8_t* os = smem + Lay::O0 + warp * Lay::OSTAGE;
 #pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
-                uint32_t o[32];
-                tmem_ld32(t_o + 32 * c, o);
-                tmem_wait_ld();
-                uint32_t wv[16];
+            for (int h = 0; h < D / 64; ++h) {
 #pragma unroll
-                for (int e = 0; e < 16; ++e)
-                    wv[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv_l, __uint_as_float(o[2 * e + 1]) * inv_l);
+                for (int c = 2 * h; c < 2 * h + 2; ++c) {
+                    uint32_t o[32];
+                    tmem_ld32(t_o + 32 * c, o);
+                    tmem_wait_ld();
+                    uint32_t wv[16];
 #pragma unroll
-                for (int v4 = 0; v4 < 4; ++v4)
-                    *reinterpret_cast<uint4*>(qs + swz_off(r, 4 * c + v4)) =
-                        make_uint4(wv[4 * v4], wv[4 * v4 + 1], wv[4 * v4 + 2], wv[4 * v4 + 3]);
+                    for (int e = 0; e < 16; ++e)
+                        wv[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv_l, __uint_as_float(o[2 * e + 1]) * inv_l);
+#pragma unroll
+                    for (int v4 = 0; v4 < 4; ++v4) {
+                        const int cc = 4 * (c - 2 * h) + v4;   // 16-byte chunk within the 64-column half
+                        *reinterpret_cast<uint4*>(os + lane * 128 + ((cc ^ (lane & 7)) << 4)) =
+                            make_uint4(wv[4 * v4], wv[4 * v4 + 1], wv[4 * v4 + 2], wv[4 * v4 + 3]);
+                    }
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    tma_store_4d(&tm_o, os, h * 64, headk, qtk * BM + (warp & 3) * 32, pw.b);
+                    bulk_commit_group();
+                    bulk_wait_group_read0();
+                }
+                __syncwarp();
             }
             tc_fence_before();
-            fence_proxy_async_smem();
-            named_barrier_sync(1 + k, 128);
-            if (r == 0) {   // rows >= L of the box are clipped by the store
-#pragma unroll
-                for (int h = 0; h < D / 64; ++h) tma_store_4d(&tm_o, qs + h * Lay::SUB, h * 64, headk, qtk * BM, pw.b);
-                bulk_commit_group();
-                bulk_wait_group_read0();
-                mbar_arrive(&sh.q_empty[k]);
-            }
 #else
             const int row = qtk * BM + r;
             uint4* dst = reinterpret_cast<uint4*>(
@@ -501,7 +524,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 for (int k = 0; k < 2 && ok; ++k) {
                     const int nk = k ? pw.n1 : pw.n0;
                     if (nk == 0) continue;
-                    // Wait until the buffer has been handed back (see GQA_EPILOGUE_TMA).
+                    // Wait until the previous pair's last S on this buffer has finished.
                     if (qn[k] > 0 && !mbar_wait(&sh.q_empty[k], (qn[k] - 1) & 1, p.err, abort)) {
                         ok = false;
                         break;
@@ -567,7 +590,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     tc_fence_after();
                     issue_s(k, ks0);
                     umma_commit(&sh.s_full[k]);
-                    if (!GQA_EPILOGUE_TMA && n[k] == 1) umma_commit(&sh.q_empty[k]);   // last S on buffer k
+                    if (n[k] == 1) umma_commit(&sh.q_empty[k]);   // that was the last S on buffer k
                 }
                 if (!ok) break;
                 umma_commit(&sh.k_empty[ks0]);
@@ -595,7 +618,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                             }
                             issue_s(k, ki % KSTAGES);
                             umma_commit(&sh.s_full[k]);
-                            if (!GQA_EPILOGUE_TMA && j + 2 == n[k]) umma_commit(&sh.q_empty[k]);
+                            if (j + 2 == n[k]) umma_commit(&sh.q_empty[k]);
                         }
                     }
                     umma_commit(&sh.v_empty[vs]);
