@@ -16,7 +16,7 @@
 //    piece of slice w and sequence b is stored in slot w + b: walking the two
 //    partitions together, every piece raises w or b by one, so slots are unique
 //    and there are at most P + B - 1 of them.
-//    Each warp owns a 3-stage ring of 16-row blocks filled by 1-D bulk copies
+//    Each warp owns a 2-stage ring of 16-row blocks filled by 1-D bulk copies
 //    (one row of K or V per lane, padded rows so ldmatrix is conflict-free).
 //    K rows are rotated in registers (RoPE on load) with cos/sin advanced by
 //    an angle-addition recurrence, re-anchored exactly every 64 blocks; the
@@ -38,10 +38,10 @@ namespace decode {
 using namespace ptx;
 
 #ifndef GQA_DECODE_STAGES
-#define GQA_DECODE_STAGES 3
+#define GQA_DECODE_STAGES 2
 #endif
 #ifndef GQA_DECODE_CTAS_PER_SM
-#define GQA_DECODE_CTAS_PER_SM 2
+#define GQA_DECODE_CTAS_PER_SM 3
 #endif
 constexpr int ROWS = 16;        // cache rows per block (MMA M)
 constexpr int NS = GQA_DECODE_STAGES;             // ring stages per warp
@@ -315,49 +315,42 @@ __global__ void __launch_bounds__(WARPS * 32, CTAS_PER_SM) split_kernel(const Pa
                 }
                 since_anchor = 0;
             }
-            // cos/sin for row t4 + 8
-            uint64_t cb[C::NP], sb[C::NP];
-#pragma unroll
-            for (int fp = 0; fp < C::NP; ++fp) {
-                const float4 r8 = rot8[(16 * (fp >> 1) + 2 * tq + 8 * (fp & 1)) >> 1];
-                cb[fp] = ca[fp];
-                sb[fp] = sa[fp];
-                rot_step(cb[fp], sb[fp], f2_pack(r8.x, r8.y), f2_pack(r8.z, r8.w));
-            }
-
             const uint32_t k_a = wsm_a + stage * C::STAGE;
             const uint32_t v_a = k_a + C::KV;
-            // ---- S^T = K' Q'^T  (M = 16 rows, N = 8 heads, K = D)
-            float sacc[4] = {0.f, 0.f, 0.f, 0.f};
+            // ---- S^T = K' Q'^T  (M = 16 rows, N = 8 heads, K = D), two independent accumulator chains.
+            // Per 16-wide step: cos/sin of row t4 + 8 from those of row t4 (one angle-addition step),
+            // rotate both rows, then advance row t4's angles to row t4 + 16 for the next block.
+            float sacc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
             const uint32_t krow = k_a + ((lane & 7) + 8 * ((lane >> 3) & 1)) * C::ROWB + 8 * (lane >> 4) * 2;
 #pragma unroll
             for (int ks = 0; ks < C::HALF_KS; ++ks) {
                 uint32_t a[4], a2[4];
                 ldsm_x4(krow + 16 * ks * 2, a[0], a[1], a[2], a[3]);
                 ldsm_x4(krow + 16 * (ks + C::HALF_KS) * 2, a2[0], a2[1], a2[2], a2[3]);
-                rot_pair(a[0], a2[0], ca[2 * ks], sa[2 * ks]);           // row t4,   dims +0,+1
-                rot_pair(a[1], a2[1], cb[2 * ks], sb[2 * ks]);           // row t4+8, dims +0,+1
-                rot_pair(a[2], a2[2], ca[2 * ks + 1], sa[2 * ks + 1]);   // row t4,   dims +8,+9
-                rot_pair(a[3], a2[3], cb[2 * ks + 1], sb[2 * ks + 1]);   // row t4+8, dims +8,+9
-                mma_bf16_16816(sacc, a[0], a[1], a[2], a[3], qb[ks][0], qb[ks][1]);
-                mma_bf16_16816(sacc, a2[0], a2[1], a2[2], a2[3], qb[ks + C::HALF_KS][0], qb[ks + C::HALF_KS][1]);
-            }
-            // advance the angles to the next block's first row (row t4 + 16)
 #pragma unroll
-            for (int fp = 0; fp < C::NP; ++fp) {
-                const float4 r8 = rot8[(16 * (fp >> 1) + 2 * tq + 8 * (fp & 1)) >> 1];
-                ca[fp] = cb[fp];
-                sa[fp] = sb[fp];
-                rot_step(ca[fp], sa[fp], f2_pack(r8.x, r8.y), f2_pack(r8.z, r8.w));
+                for (int hf = 0; hf < 2; ++hf) {   // dims 16ks + 2tq + 8*hf + {0, 1}
+                    const int fp = 2 * ks + hf;
+                    const float4 r8 = rot8[(16 * ks + 2 * tq + 8 * hf) >> 1];
+                    const uint64_t Cr = f2_pack(r8.x, r8.y), Sr = f2_pack(r8.z, r8.w);
+                    uint64_t cb = ca[fp], sb = sa[fp];
+                    rot_step(cb, sb, Cr, Sr);                       // row t4 + 8
+                    rot_pair(a[2 * hf], a2[2 * hf], ca[fp], sa[fp]);          // row t4
+                    rot_pair(a[2 * hf + 1], a2[2 * hf + 1], cb, sb);          // row t4 + 8
+                    ca[fp] = cb;
+                    sa[fp] = sb;
+                    rot_step(ca[fp], sa[fp], Cr, Sr);               // row t4 + 16: next block's first row
+                }
+                mma_bf16_16816(sacc[0], a[0], a[1], a[2], a[3], qb[ks][0], qb[ks][1]);
+                mma_bf16_16816(sacc[1], a2[0], a2[1], a2[2], a2[3], qb[ks + C::HALF_KS][0], qb[ks + C::HALF_KS][1]);
             }
             ++since_anchor;
 
             // ---- online softmax over the block (heads 2tq, 2tq+1 per lane; rows t4, t4+8)
             const bool v_lo = t4 < nvalid, v_hi = t4 + 8 < nvalid;
-            const float x0 = v_lo ? sacc[0] * sl2 : -INFINITY;
-            const float x1 = v_lo ? sacc[1] * sl2 : -INFINITY;
-            const float x2 = v_hi ? sacc[2] * sl2 : -INFINITY;
-            const float x3 = v_hi ? sacc[3] * sl2 : -INFINITY;
+            const float x0 = v_lo ? (sacc[0][0] + sacc[1][0]) * sl2 : -INFINITY;
+            const float x1 = v_lo ? (sacc[0][1] + sacc[1][1]) * sl2 : -INFINITY;
+            const float x2 = v_hi ? (sacc[0][2] + sacc[1][2]) * sl2 : -INFINITY;
+            const float x3 = v_hi ? (sacc[0][3] + sacc[1][3]) * sl2 : -INFINITY;
             float bm0 = fmaxf(x0, x2), bm1 = fmaxf(x1, x3);
 #pragma unroll
             for (int sh = 4; sh < 32; sh <<= 1) {
