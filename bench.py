@@ -276,7 +276,7 @@ def run_ours(args):
     import grouped_query_attention_gqa_b200 as G
     G.load()
 
-    wp = gi.BY_NAME[PREFILL_WORKLOAD]
+    wp = gi.BY_NAME[args.prefill_workload]
     wd = gi.BY_NAME[DECODE_WORKLOAD]
     if args.decode_batch:
         wd = wd.with_(B=args.decode_batch, desc=wd.desc.replace("B=64", f"B={args.decode_batch}"))
@@ -402,7 +402,7 @@ def run_ours(args):
             "roofline": {"kernel": "attn_kernel (prefill)", "bound": "tensor", "achieved": achieved_t,
                          "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved_t / peaks["bf16_tflops"],
                          "peak_source": f"{peak_src} bf16 dense (burst)",
-                         "traffic": profile_traffic("attn_kernel", PREFILL_WORKLOAD),
+                         "traffic": profile_traffic("attn_kernel", wp.name),
                          "algorithmic_flops_per_launch": fl, "ms_per_launch": attn_mean},
             "cpu_baseline": cpu_baseline(wp) if (world == 1 and not args.no_cpu_baseline) else None,
             "only": args.only,
@@ -447,6 +447,8 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffer) leg")
     ap.add_argument("--only", choices=["prefill", "decode"], default=None,
                     help="run one half of the step only (profiling; the line then carries that half)")
+    ap.add_argument("--prefill-workload", default=PREFILL_WORKLOAD, choices=[w.name for w in gi.WORKLOADS if w.kind == "prefill"],
+                    help="prefill workload of the step (default: the Qwen2-7B L=4096 headline workload)")
     ap.add_argument("--decode-batch", type=int, default=None,
                     help="decode with this many sequences instead of 64 (smaller profiling case)")
     args = ap.parse_args(argv)
