@@ -65,8 +65,8 @@ constexpr int OTHER_REGS = 80;
 static_assert(256 * SOFTMAX_REGS + 128 * OTHER_REGS <= NUM_THREADS * LAUNCH_REGS, "register split");
 constexpr uint32_t TMEM_COLS = 512;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: O is rescaled only when the max grows by > 2^8
-// Of every 8 consecutive exponentials of a row (off the diagonal tile), this many run on the FMA
-// pipe (exp2_poly) and the rest on the ex2 unit.
+// Of every 8 consecutive pairs of exponentials of a row (off the diagonal tile), this many run on
+// the FMA pipe (exp2_poly_x2) and the rest on the ex2 unit.
 #ifndef GQA_EXP_POLY_OF_8
 #define GQA_EXP_POLY_OF_8 1
 #endif
@@ -227,28 +227,32 @@ __device__ __forceinline__ uint32_t pack_p(float lo, float hi) {
 // with masked entries, whose weights must be exactly 0).
 template <bool POLY>
 __device__ __forceinline__ float row_exp_store(const uint32_t (&sr)[4][32], float sl2, float neg_m, uint32_t t_s) {
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    const uint64_t scale2 = f2_pack(sl2, sl2), shift2 = f2_pack(neg_m, neg_m);
+    uint64_t acc[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
-            const float x0 = fmaf(__uint_as_float(sr[c][e]), sl2, neg_m);
-            const float x1 = fmaf(__uint_as_float(sr[c][e + 1]), sl2, neg_m);
-            const float p0 = (POLY && (e & 7) < GQA_EXP_POLY_OF_8) ? exp2_poly(x0) : ex2(x0);
-            const float p1 = (POLY && ((e + 1) & 7) < GQA_EXP_POLY_OF_8) ? exp2_poly(x1) : ex2(x1);
-#if GQA_PACK_TRUNC
-            const uint32_t b0 = __float_as_uint(p0), b1 = __float_as_uint(p1);
-            pk[e >> 1] = __byte_perm(b0, b1, 0x7632);
-            acc[(e >> 1) & 3] += __uint_as_float(b0 & 0xFFFF0000u) + __uint_as_float(b1 & 0xFFFF0000u);
-#else
-            acc[(e >> 1) & 3] += p0 + p1;
+            const uint64_t x = f2_fma(f2_pack(__uint_as_float(sr[c][e]), __uint_as_float(sr[c][e + 1])), scale2, shift2);
+            float p0, p1;
+            if (POLY && ((e >> 1) & 7) < GQA_EXP_POLY_OF_8) {
+                exp2_poly_x2(x, p0, p1);
+            } else {
+                float x0, x1;
+                f2_unpack(x, x0, x1);
+                p0 = ex2(x0);
+                p1 = ex2(x1);
+            }
+            acc[(e >> 1) & 1] = f2_add(acc[(e >> 1) & 1], f2_pack(p0, p1));
             pk[e >> 1] = pack_p(p0, p1);
-#endif
         }
         tmem_st16(t_s + 16 * c, pk);
     }
-    return (acc[0] + acc[1]) + (acc[2] + acc[3]);
+    float a0, a1, b0, b1;
+    f2_unpack(acc[0], a0, a1);
+    f2_unpack(acc[1], b0, b1);
+    return (a0 + a1) + (b0 + b1);
 }
 
 // Byte address of 16-byte chunk `cc` (8 bf16 along d) of row r in a K-major, 128-byte-swizzled tile.
@@ -372,13 +376,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                         for (int e = 0; e < 32; ++e)
                             if (32 * c + e > r) sr[c][e] = __float_as_uint(-INFINITY);
                 }
-                float mxs[8];   // eight independent running maxima instead of one serial chain
+                float mxs[8];   // eight independent running maxima, two scores per 3-input max
 #pragma unroll
                 for (int e = 0; e < 8; ++e) mxs[e] = __uint_as_float(sr[0][e]);
 #pragma unroll
-                for (int i = 8; i < 128; ++i) mxs[i & 7] = fmaxf(mxs[i & 7], __uint_as_float(sr[i >> 5][i & 31]));
-                const float mx = fmaxf(fmaxf(fmaxf(mxs[0], mxs[1]), fmaxf(mxs[2], mxs[3])),
-                                       fmaxf(fmaxf(mxs[4], mxs[5]), fmaxf(mxs[6], mxs[7])));
+                for (int i = 8; i < 128; i += 2)
+                    mxs[(i >> 1) & 7] = fmax3(mxs[(i >> 1) & 7], __uint_as_float(sr[i >> 5][i & 31]),
+                                              __uint_as_float(sr[i >> 5][(i & 31) + 1]));
+                const float mx = fmaxf(fmax3(mxs[0], mxs[1], mxs[2]), fmax3(fmax3(mxs[3], mxs[4], mxs[5]), mxs[6], mxs[7]));
                 const float m_new = fmaxf(m_run, mx * sl2);
                 if (j == 0) {
                     m_run = m_new;

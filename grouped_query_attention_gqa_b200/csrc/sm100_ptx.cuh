@@ -276,31 +276,7 @@ __device__ __forceinline__ void regs_decrease() {
 }
 
 // ----------------------------------------------------------------------------
-// Fast base-2 exponential (the hardware ex2 instruction; ~2 ulp, flushes denormals).
-__device__ __forceinline__ float ex2(float x) {
-    float y;
-    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
-
-// 2^x on the FMA pipe, for part of the softmax exponentials (the ex2 unit is the co-bottleneck
-// with the tensor core at d = 128).  Range reduction 2^x = 2^n * 2^f, n = round(x), f in [-1/2, 1/2]:
-// adding 1.5 * 2^23 leaves round(x) in the low mantissa bits; 2^f is a degree-3 polynomial fitted by
-// the Remez exchange algorithm for minimum relative error on [-1/2, 1/2] (7.5e-5, far below the
-// bf16 rounding of P); 2^n is added to the exponent field.  x is clamped to [-125, inf) so the
-// exponent never underflows: callers must not rely on an exact 0 for x = -inf (masked entries).
-__device__ __forceinline__ float exp2_poly(float x) {
-    x = fmaxf(x, -125.0f);
-    const float t = x + 12582912.0f;
-    const float r = t - 12582912.0f;
-    const float f = x - r;
-    float p = fmaf(f, 0.0551716685f, 0.2426111251f);
-    p = fmaf(p, f, 0.6932609677f);
-    p = fmaf(p, f, 0.9999280572f);
-    const int n = __float_as_int(t) - 0x4B400000;
-    return __int_as_float(__float_as_int(p) + (n << 23));
-}
-
+// bf16 packing and unpacking.
 // Two fp32 -> packed bf16x2 (round to nearest even); `lo` lands in the low half.
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     uint32_t r;
@@ -334,6 +310,11 @@ __device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
     asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
     return d;
 }
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
 __device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
     uint64_t d;
     asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
@@ -353,6 +334,60 @@ __device__ __forceinline__ uint32_t f2_to_bf16x2(uint64_t v) {
     f2_unpack(v, lo, hi);
     return pack_bf16x2(lo, hi);
 }
+
+// ----------------------------------------------------------------------------
+// Fast base-2 exponential (the hardware ex2 instruction; ~2 ulp, flushes denormals).
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// 2^x on the FMA pipe, for part of the softmax exponentials (the ex2 unit is the co-bottleneck
+// with the tensor core at d = 128).  Range reduction 2^x = 2^n * 2^f, n = round(x), f in [-1/2, 1/2]:
+// adding 1.5 * 2^23 leaves round(x) in the low mantissa bits; 2^f is a degree-3 polynomial fitted by
+// the Remez exchange algorithm for minimum relative error on [-1/2, 1/2] (7.5e-5, far below the
+// bf16 rounding of P); 2^n is added to the exponent field.  x is clamped to [-125, inf) so the
+// exponent never underflows: callers must not rely on an exact 0 for x = -inf (masked entries).
+__device__ __forceinline__ float exp2_poly(float x) {
+    x = fmaxf(x, -125.0f);
+    const float t = x + 12582912.0f;
+    const float r = t - 12582912.0f;
+    const float f = x - r;
+    float p = fmaf(f, 0.0551716685f, 0.2426111251f);
+    p = fmaf(p, f, 0.6932609677f);
+    p = fmaf(p, f, 0.9999280572f);
+    const int n = __float_as_int(t) - 0x4B400000;
+    return __int_as_float(__float_as_int(p) + (n << 23));
+}
+
+// 2^x for an fp32 pair (lo, hi) on the FMA pipe: the same range reduction and polynomial as
+// exp2_poly, done with paired instructions.  (t << 23) equals (n << 23) modulo 2^32 because the low
+// nine bits of the bias 0x4B400000 are zero, so the exponent add needs no bias subtraction.
+__device__ __forceinline__ void exp2_poly_x2(uint64_t xx, float& y0, float& y1) {
+    float x0, x1;
+    f2_unpack(xx, x0, x1);
+    const uint64_t magic = f2_pack(12582912.0f, 12582912.0f);
+    const uint64_t x = f2_pack(fmaxf(x0, -125.0f), fmaxf(x1, -125.0f));
+    const uint64_t t = f2_add(x, magic);
+    const uint64_t f = f2_sub(x, f2_sub(t, magic));
+    uint64_t p = f2_fma(f, f2_pack(0.0551716685f, 0.0551716685f), f2_pack(0.2426111251f, 0.2426111251f));
+    p = f2_fma(p, f, f2_pack(0.6932609677f, 0.6932609677f));
+    p = f2_fma(p, f, f2_pack(0.9999280572f, 0.9999280572f));
+    float p0, p1, t0, t1;
+    f2_unpack(p, p0, p1);
+    f2_unpack(t, t0, t1);
+    y0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
+    y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
+}
+
+// max(a, b, c) in one instruction (sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
 
 // ----------------------------------------------------------------------------
 // Legacy warp-level tensor-core path (decode).
