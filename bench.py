@@ -1,7 +1,7 @@
 #!/usr/bin/env python
 """Benchmark of the GQA hot path on B200: prefill TFLOP/s and decode KV-cache GB/s.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference|flashinfer]
     torchrun --nproc-per-node N bench.py --gpus N ...      (one process per GPU)
 
 One step is one pass of the whole hot path: a causal prefill over the Qwen2-7B-shaped workload
@@ -16,6 +16,7 @@ the workload (independent batches, no collective on the data path: weak scaling)
 
 `--impl reference` times the plain fp64 CPU oracle (the only reference that exists for this
 method) on a bounded sample of the same prefill workload, on the host cores of rank 0.
+`--impl flashinfer` times installed library attention kernels on the prefill workload, for context.
 """
 from __future__ import annotations
 
@@ -257,6 +258,77 @@ def run_reference(args):
     return 0
 
 
+# ------------------------------------------------------------------------------ library context arm
+def run_library(args):
+    """Time flashinfer's Blackwell attention kernels on the prefill workload (context, not a target).
+
+    Plain causal GQA attention on the same shape, inputs, FLOP count and L2 flush as the prefill of
+    `--impl ours`, without RoPE: compare its TFLOP/s with the `roofline.achieved` of our attention
+    kernel.  Backends: "trtllm-gen" (TensorRT-LLM FMHA, precompiled), "cutlass" (CUTLASS sm100 FMHA,
+    compiled on first use, about two minutes), "cute-dsl" (CuTe DSL kernel).  Rank 0 only.
+    """
+    rank, local, _ = dist_env()
+    if rank != 0:
+        return 0
+    import flashinfer
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    w = gi.BY_NAME[args.prefill_workload]
+    B, L, hq, hkv, d = w.B, w.L, w.h_q, w.h_kv, w.d
+    q4, k4, v4 = gi.prefill_inputs(w, device=str(dev))
+    q, k, v = q4.reshape(B * L, hq, d), k4.reshape(B * L, hkv, d), v4.reshape(B * L, hkv, d)
+    indptr = torch.arange(0, (B + 1) * L, L, dtype=torch.int32, device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    fl = prefill_flops(w)
+    results = {}
+    for backend in args.library_backends.split(","):
+        ws = torch.zeros(256 << 20, dtype=torch.uint8, device=dev)
+        if backend == "trtllm-gen":
+            page = 64
+            npg = (L + page - 1) // page
+            pad = npg * page - L
+            def paged(x):
+                x = torch.nn.functional.pad(x.reshape(B, L, hkv, d), (0, 0, 0, 0, 0, pad))
+                return x.view(B, npg, page, hkv, d).permute(0, 1, 3, 2, 4).reshape(B * npg, hkv, page, d).contiguous()
+            kc, vc = paged(k), paged(v)
+            bt = torch.arange(B * npg, dtype=torch.int32, device=dev).view(B, npg)
+            sl = torch.full((B,), L, dtype=torch.int32, device=dev)
+            o = torch.empty_like(q)
+            fn = lambda: flashinfer.prefill.trtllm_batch_context_with_kv_cache(
+                q, (kc, vc), ws, bt, sl, L, L, 1.0 / d ** 0.5, 1.0, B, indptr, indptr, out=o,
+                kv_layout="HND", causal=True)
+        else:
+            wr = flashinfer.BatchPrefillWithRaggedKVCacheWrapper(ws, "NHD", backend=backend)
+            wr.plan(indptr, indptr, hq, hkv, d, causal=True, q_data_type=torch.bfloat16,
+                    kv_data_type=torch.bfloat16)
+            fn = lambda: wr.run(q, k, v)
+        for _ in range(args.warmup):
+            fn()
+        ms = []
+        for _ in range(args.steps):
+            flush.zero_()
+            a, b = ev(), ev()
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize()
+            ms.append(a.elapsed_time(b))
+        mean = sum(ms) / len(ms)
+        results[backend] = {"ms_per_launch": mean, "tflops": fl / mean / 1e9}
+    best = max(results, key=lambda b_: results[b_]["tflops"])
+    peaks, src = load_peaks()
+    line = {"metric": METRIC, "value": results[best]["tflops"], "unit": "TFLOP/s", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": results[best]["ms_per_launch"],
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic", "config": dict(bench_config(w, gi.BY_NAME[DECODE_WORKLOAD]),
+                                                 step="attention kernel only, no RoPE, L2 flushed before each launch"),
+            "impl": "flashinfer", "flashinfer_version": flashinfer.__version__, "best_backend": best,
+            "frac_of_bf16_peak": results[best]["tflops"] / peaks["bf16_tflops"], "peak_source": src,
+            "backends": results}
+    print(json.dumps(clean(line)), flush=True)
+    return 0
+
+
 # ------------------------------------------------------------------------------------------ GPU arm
 def ev():
     e = torch.cuda.Event(enable_timing=True)
@@ -286,12 +358,22 @@ def run_ours(args):
     else:   # placeholders of the right shape; the prefill does not run
         q, k, v = (torch.empty(1, 1, 1, 8, dtype=torch.bfloat16, device=dev) for _ in range(3))
     out = torch.empty_like(q)
-    if do_d:
+    page = args.decode_page_size
+    table = None
+    if do_d and page:   # the same logical cache, scattered over pages of `page` rows
+        s, qd, kc, vc, table, _, _, _ = gi.decode_paged_inputs(wd, page, device=str(dev))
+    elif do_d:
         s, qd, kc, vc = gi.decode_inputs(wd, device=str(dev))
     else:
         s = torch.ones(1, dtype=torch.int32, device=dev)
         qd, kc, vc = (torch.empty(1, 1, 8, dtype=torch.bfloat16, device=dev) for _ in range(3))
     outd = torch.empty_like(qd)
+
+    def dec_call(qx, sx, tx):
+        if tx is None:
+            G.decode(qx, kc, vc, sx, theta=wd.theta, out=outd)
+        else:
+            G.decode_paged(qx, kc, vc, tx, sx, theta=wd.theta, out=outd)
     total_rows = int(s.sum().item())
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     K, W = args.steps, args.warmup
@@ -307,7 +389,7 @@ def run_ours(args):
             evs[3].record()
             G.set_timing_events(evs[4], evs[5])
         if do_d:
-            G.decode(qd, kc, vc, s, theta=wd.theta, out=outd)
+            dec_call(qd, s, table)
         if evs:
             evs[6].record()
             G.set_timing_events(None, None)
@@ -353,6 +435,8 @@ def run_ours(args):
         qdh, sh_ = qd.cpu().pin_memory(), s.cpu().pin_memory()
         outdh = torch.empty(outd.shape, dtype=outd.dtype).pin_memory()
         qx, kx, vx, qdx, sx = (torch.empty_like(x) for x in (q, k, v, qd, s))
+        th = table.cpu().pin_memory() if table is not None else None
+        tx = torch.empty_like(table) if table is not None else None
 
     def e2e_step(e):
         flush.zero_()
@@ -365,7 +449,9 @@ def run_ours(args):
         e[1].record()
         qdx.copy_(qdh, non_blocking=True)
         sx.copy_(sh_, non_blocking=True)
-        G.decode(qdx, kc, vc, sx, theta=wd.theta, out=outd)
+        if tx is not None:
+            tx.copy_(th, non_blocking=True)
+        dec_call(qdx, sx, tx)
         outdh.copy_(outd, non_blocking=True)
         e[2].record()
 
@@ -413,18 +499,21 @@ def run_ours(args):
             "clocks": sampler.summary(),
             "decode": {
                 "workload": wd.desc, "total_cache_rows": total_rows,
+                "layout": f"paged: {page} rows per page, pages scattered in a seeded random order" if page
+                          else "packed",
                 "value": world * allb / (dec_mean * 1e-3) / 1e9, "unit": "GB/s",
                 "kv_gbs": world * kvb / (dec_mean * 1e-3) / 1e9,
                 "ms_per_step": dec_mean,
                 "roofline": {"kernel": "split_kernel (decode)", "bound": "hbm", "achieved": achieved_b,
                              "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": achieved_b / peaks["hbm_gbs"],
                              "peak_source": f"{peak_src} HBM copy",
-                             "traffic": profile_traffic("split_kernel", DECODE_WORKLOAD),
+                             "traffic": profile_traffic("split_kernel", DECODE_WORKLOAD + (f"-paged{page}" if page else "")),
                              "algorithmic_bytes_per_launch": allb, "ms_per_launch": split_mean},
                 "e2e": {"value": world * allb / (e2e_dec * 1e-3) / 1e9, "unit": "GB/s",
-                        "h2d_bytes_per_step": qd.numel() * 2 + s.numel() * 4,
+                        "h2d_bytes_per_step": qd.numel() * 2 + s.numel() * 4 + (table.numel() * 4 if page else 0),
                         "d2h_bytes_per_step": outd.numel() * 2,
-                        "note": "the KV cache is resident device state; the step's inputs are q and the lengths"},
+                        "note": "the KV cache is resident device state; the step's inputs are q, the lengths"
+                                + (" and the block table" if page else "")},
             },
             "wall_s_timed_region": t_wall,
             "impl": "ours",
@@ -442,13 +531,19 @@ def main(argv=None):
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--impl", choices=["ours", "reference", "flashinfer"], default="ours",
+                    help="ours: the CUDA path; reference: the fp64 oracle on the host; flashinfer: library "
+                         "attention kernels on the prefill workload, for context")
+    ap.add_argument("--library-backends", default="trtllm-gen",
+                    help="flashinfer backends timed by --impl flashinfer (comma list of trtllm-gen, cutlass, cute-dsl)")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the host oracle timing")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffer) leg")
     ap.add_argument("--only", choices=["prefill", "decode"], default=None,
                     help="run one half of the step only (profiling; the line then carries that half)")
     ap.add_argument("--prefill-workload", default=PREFILL_WORKLOAD, choices=[w.name for w in gi.WORKLOADS if w.kind == "prefill"],
                     help="prefill workload of the step (default: the Qwen2-7B L=4096 headline workload)")
+    ap.add_argument("--decode-page-size", type=int, default=None,
+                    help="decode through gqa_decode_paged, the cache in pages of this many rows")
     ap.add_argument("--decode-batch", type=int, default=None,
                     help="decode with this many sequences instead of 64 (smaller profiling case)")
     args = ap.parse_args(argv)
@@ -456,6 +551,8 @@ def main(argv=None):
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
         return run_reference(args)
+    if args.impl == "flashinfer":
+        return run_library(args)
     return run_ours(args)
 
 

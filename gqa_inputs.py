@@ -113,6 +113,51 @@ def decode_inputs(w: Workload, device: str = "cpu", seqlens=None):
     return drawn, q, kc, vc
 
 
+def paged_layout(seqlens, page_size: int, seed: int, extra_pages: int = 3, max_pages: int | None = None,
+                 device: str = "cpu"):
+    """A seeded paged placement of sequences of the given lengths (storage layout only).
+
+    Each sequence b needs ceil(seqlens[b] / page_size) pages; all needed pages plus `extra_pages`
+    unused ones are numbered in a random order, so neighbouring pages of a sequence are scattered.
+    Returns (block_table int32 [B, max_pages], num_pages, store_row int64 [sum(seqlens)]), where
+    block_table[b, i] is the page of the i-th block of sequence b (-1 past its last page) and
+    store_row[off_b + j] = page * page_size + j % page_size is where packed row off_b + j lives.
+    """
+    lens = [int(x) for x in torch.as_tensor(seqlens).tolist()]
+    need = [(n + page_size - 1) // page_size for n in lens]
+    num_pages = sum(need) + extra_pages
+    mp = max(need + [1]) if max_pages is None else max_pages
+    perm = torch.randperm(num_pages, generator=_gen(seed, "cpu")).to(torch.int32)
+    table = torch.full((len(lens), mp), -1, dtype=torch.int32)
+    rows = []
+    nxt = 0
+    for b, (n, k) in enumerate(zip(lens, need)):
+        table[b, :k] = perm[nxt:nxt + k]
+        nxt += k
+        j = torch.arange(n, dtype=torch.int64)
+        rows.append(table[b, (j // page_size)].to(torch.int64) * page_size + j % page_size)
+    store_row = torch.cat(rows) if rows else torch.zeros(0, dtype=torch.int64)
+    return table.to(device), num_pages, store_row.to(device)
+
+
+def decode_paged_inputs(w: Workload, page_size: int, device: str = "cpu", seqlens=None, extra_pages: int = 3):
+    """decode_inputs(w) with the packed caches scattered into pages.
+
+    Returns seqlens, q, kpages, vpages [num_pages, page_size, h_kv, d], block_table [B, max_pages],
+    num_pages, and the packed caches themselves.  Page slots that hold no cache row are filled with
+    N(0,1) values, so a wrong slot read shows up in the result.
+    """
+    s, q, kc, vc = decode_inputs(w, device, seqlens=seqlens)
+    table, num_pages, store_row = paged_layout(s.cpu(), page_size, w.seed + 7919, extra_pages, device=device)
+    gen = _gen(w.seed + 104729, device)
+    kp = _randn_bf16((num_pages * page_size, w.h_kv, w.d), gen, device)
+    vp = _randn_bf16((num_pages * page_size, w.h_kv, w.d), gen, device)
+    kp[store_row] = kc
+    vp[store_row] = vc
+    shape = (num_pages, page_size, w.h_kv, w.d)
+    return s, q, kp.view(shape), vp.view(shape), table, num_pages, kc, vc
+
+
 def small(kind: str, B: int, h_q: int, h_kv: int, d: int, L: int = 0, max_len: int = 0,
           seed: int = 7, theta: float = THETA, name: str = "") -> Workload:
     """A small ad-hoc workload for tests (ragged sizes, special head counts)."""

@@ -4,5 +4,6 @@ The computation lives in libgqa.so (hand-written sm_100a CUDA behind the C ABI o
 include/gqa.h); this package is its thin Python binding.
 """
 from ._lib import (  # noqa: F401
-    GQAError, DEVERR_SEQLEN, DEVERR_TIMEOUT, LIB_PATH, decode, last_error, load, prefill, release, set_timing_events, strerror,
+    GQAError, DEVERR_PAGE, DEVERR_SEQLEN, DEVERR_TIMEOUT, LIB_PATH, decode, decode_paged, last_error, load, prefill,
+    release, set_timing_events, strerror,
 )

@@ -18,6 +18,7 @@ LIB_PATH = os.path.join(_PKG, "libgqa.so")
 GQA_OK = 0
 DEVERR_SEQLEN = 1
 DEVERR_TIMEOUT = 2
+DEVERR_PAGE = 4
 
 _lib = None
 
@@ -42,6 +43,8 @@ def load() -> ctypes.CDLL:
     lib.gqa_prefill.restype = i
     lib.gqa_decode.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f]
     lib.gqa_decode.restype = i
+    lib.gqa_decode_paged.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, f]
+    lib.gqa_decode_paged.restype = i
     lib.gqa_set_timing_events.argtypes = [vp, vp]
     lib.gqa_set_timing_events.restype = i
     lib.gqa_set_stream.argtypes = [vp]
@@ -124,6 +127,38 @@ def decode(q: torch.Tensor, kcache: torch.Tensor, vcache: torch.Tensor, seqlens:
                                B, h_q, h_kv, d, float(theta))
     if rc != GQA_OK:
         raise GQAError(rc, "gqa_decode")
+    return out
+
+
+def decode_paged(q: torch.Tensor, kpages: torch.Tensor, vpages: torch.Tensor, block_table: torch.Tensor,
+                 seqlens: torch.Tensor, theta: float = 1.0e6, out: torch.Tensor | None = None) -> torch.Tensor:
+    """One decode step over a paged cache.
+
+    q [B, h_q, d]; kpages / vpages [num_pages, page_size, h_kv, d]; block_table int32 [B, max_pages]
+    (device): position j of sequence b is slot j % page_size of page block_table[b, j // page_size];
+    seqlens int32 [B] (device).
+    """
+    if q.dim() != 3 or kpages.dim() != 4:
+        raise ValueError("q must be [B, h_q, d] and kpages [num_pages, page_size, h_kv, d]")
+    B, h_q, d = q.shape
+    num_pages, page_size, h_kv = kpages.shape[:3]
+    _check(q, "q", None)
+    _check(kpages, "kpages", (num_pages, page_size, h_kv, d))
+    _check(vpages, "vpages", tuple(kpages.shape))
+    _check(seqlens, "seqlens", (B,), dtype=torch.int32)
+    if block_table.dim() != 2 or block_table.shape[0] != B:
+        raise ValueError(f"block_table must be [B={B}, max_pages], got {tuple(block_table.shape)}")
+    _check(block_table, "block_table", None, dtype=torch.int32)
+    if out is None:
+        out = torch.empty_like(q)
+    _check(out, "out", (B, h_q, d))
+    with torch.cuda.device(q.device):
+        _stream(q.device)
+        rc = load().gqa_decode_paged(_ptr(q), _ptr(kpages), _ptr(vpages), _ptr(block_table), _ptr(seqlens),
+                                     _ptr(out), B, h_q, h_kv, d, page_size, num_pages, block_table.shape[1],
+                                     float(theta))
+    if rc != GQA_OK:
+        raise GQAError(rc, "gqa_decode_paged")
     return out
 
 

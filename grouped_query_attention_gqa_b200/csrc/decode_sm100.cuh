@@ -68,8 +68,10 @@ struct Cfg {
 
 struct Params {
     const __nv_bfloat16* q;    // [B, h_q, D]
-    const __nv_bfloat16* kc;   // [N, h_kv, D]
-    const __nv_bfloat16* vc;   // [N, h_kv, D]
+    const __nv_bfloat16* kc;   // packed: [N, h_kv, D]; paged: [num_pages * page_size, h_kv, D]
+    const __nv_bfloat16* vc;   // same layout as kc
+    const int* bt;             // paged only: block table [B, max_pages]; nullptr for the packed layout
+    int page_size, max_pages, num_pages;
     __nv_bfloat16* out;        // [B, h_q, D]
     const int64_t* off;        // [B + 1] packed row offsets
     float* part;               // [(P + B) * h_kv * n_hb * PART]
@@ -235,14 +237,32 @@ __global__ void __launch_bounds__(WARPS * 32, CTAS_PER_SM) split_kernel(const Pa
     auto issue = [&](int stage) {
         const int nvalid = static_cast<int>(iss.seg_end - iss.r < ROWS ? iss.seg_end - iss.r : ROWS);
         uint64_t* bar = &bars[warp][stage];
-        if (lane == 0) mbar_arrive_expect_tx(bar, static_cast<uint32_t>(nvalid * D * 2 * 2));
-        __syncwarp();
         const int i = lane & (ROWS - 1);
         const bool is_v = lane >= ROWS;
+        // Storage row of logical row iss.r + i: the packed row itself, or its page slot through the block
+        // table.  A table entry outside [0, num_pages), or a row past max_pages pages, is not read: the
+        // row stays zero and the device error word gets kErrBadPage.
+        bool load = i < nvalid;
+        int64_t srow = iss.r + i;
+        if (load && p.bt) {
+            const int j = static_cast<int>(srow - p.off[iss.b]);   // position in the sequence (< 2^31)
+            const int pi = j / p.page_size;
+            const int page = pi < p.max_pages ? p.bt[static_cast<int64_t>(iss.b) * p.max_pages + pi] : -1;
+            if (page < 0 || page >= p.num_pages) {
+                load = false;
+                atomicOr(p.err, kErrBadPage);
+            } else {
+                srow = static_cast<int64_t>(page) * p.page_size + (j - pi * p.page_size);
+            }
+        }
+        // Arm the stage with the bytes of the rows that are really copied.
+        const uint32_t nload = __popc(__ballot_sync(0xffffffffu, load));
+        if (lane == 0) mbar_arrive_expect_tx(bar, nload * static_cast<uint32_t>(D * 2));
+        __syncwarp();
         uint8_t* dst = wsm + stage * C::STAGE + (is_v ? C::KV : 0) + i * C::ROWB;
         fence_proxy_async_smem();
-        if (i < nvalid) {
-            const __nv_bfloat16* src = (is_v ? p.vc : p.kc) + (iss.r + i) * row_stride + static_cast<size_t>(u) * D;
+        if (load) {
+            const __nv_bfloat16* src = (is_v ? p.vc : p.kc) + srow * row_stride + static_cast<size_t>(u) * D;
             bulk_load(dst, src, D * 2, bar);
         } else {
 #pragma unroll

@@ -202,9 +202,11 @@ int launch_prefill(DeviceState* st, const void* q, const void* k, const void* v,
     return GQA_OK;
 }
 
+// Packed cache (bt == nullptr) or paged cache through the block table bt [B, max_pages].
 template <int D>
 int launch_decode(DeviceState* st, const void* q, const void* kc, const void* vc, const int* seqlens, void* out,
-                  int B, int h_q, int h_kv, float theta) {
+                  int B, int h_q, int h_kv, float theta, const int* bt = nullptr, int page_size = 0,
+                  int num_pages = 0, int max_pages = 0) {
     using namespace gqa::decode;
     using C = Cfg<D>;
     const int g = h_q / h_kv;
@@ -222,6 +224,10 @@ int launch_decode(DeviceState* st, const void* q, const void* kc, const void* vc
     p.kc = static_cast<const __nv_bfloat16*>(kc);
     p.vc = static_cast<const __nv_bfloat16*>(vc);
     p.out = static_cast<__nv_bfloat16*>(out);
+    p.bt = bt;
+    p.page_size = page_size;
+    p.num_pages = num_pages;
+    p.max_pages = max_pages;
     p.off = static_cast<int64_t*>(st->dws);
     p.part = reinterpret_cast<float*>(static_cast<uint8_t*>(st->dws) + off_bytes);
     p.B = B;
@@ -297,6 +303,8 @@ int launch_decode_fixed_scratch(DeviceState* st, const void* q, const void* kc, 
     p.kc = static_cast<const __nv_bfloat16*>(kc);
     p.vc = static_cast<const __nv_bfloat16*>(vc);
     p.out = static_cast<__nv_bfloat16*>(out);
+    p.bt = nullptr;
+    p.page_size = p.num_pages = p.max_pages = 0;
     p.off = static_cast<int64_t*>(st->fixed_scratch);
     p.part = reinterpret_cast<float*>(static_cast<uint8_t*>(st->fixed_scratch) + off_bytes);
     p.B = B;
@@ -398,6 +406,26 @@ int gqa_decode_noalloc(const void* q, const void* kcache, const void* vcache, co
     if (!st) return rc;
     return d == 64 ? launch_decode_fixed_scratch<64>(st, q, kcache, vcache, seqlens, out, B, h_q, h_kv, theta)
                    : launch_decode_fixed_scratch<128>(st, q, kcache, vcache, seqlens, out, B, h_q, h_kv, theta);
+}
+
+int gqa_decode_paged(const void* q, const void* kpages, const void* vpages, const int* block_table,
+                     const int* seqlens, void* out, int B, int h_q, int h_kv, int d, int page_size, int num_pages,
+                     int max_pages_per_seq, float theta) {
+    if (B < 0 || page_size <= 0 || num_pages <= 0 || max_pages_per_seq <= 0) return GQA_ERR_DIMS;
+    // Storage rows are indexed page * page_size + slot in 64 bits; positions stay below 2^31.
+    if (static_cast<long long>(num_pages) * page_size > (1LL << 40)) return GQA_ERR_DIMS;
+    if (static_cast<long long>(B) * max_pages_per_seq > 0x7fffffffLL) return GQA_ERR_DIMS;
+    int rc = check_common(h_q, h_kv, d, theta);
+    if (rc != GQA_OK) return rc;
+    if (B == 0) return GQA_OK;
+    if (!q || !kpages || !vpages || !block_table || !seqlens || !out) return GQA_ERR_NULL;
+    if (!aligned16(q) || !aligned16(kpages) || !aligned16(vpages) || !aligned16(out)) return GQA_ERR_ALIGN;
+    DeviceState* st = device_state(&rc);
+    if (!st) return rc;
+    return d == 64 ? launch_decode<64>(st, q, kpages, vpages, seqlens, out, B, h_q, h_kv, theta, block_table,
+                                       page_size, num_pages, max_pages_per_seq)
+                   : launch_decode<128>(st, q, kpages, vpages, seqlens, out, B, h_q, h_kv, theta, block_table,
+                                        page_size, num_pages, max_pages_per_seq);
 }
 
 int gqa_last_error(void) {

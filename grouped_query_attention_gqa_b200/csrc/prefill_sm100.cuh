@@ -85,8 +85,17 @@ constexpr float kRescaleThreshold = 8.0f;   // log2 units: O is rescaled only wh
 #ifndef GQA_EPILOGUE_TMA
 #define GQA_EPILOGUE_TMA 1
 #endif
-constexpr int PREP_POS = 8;                 // positions per CTA of the prep kernel
-constexpr int PREP_UNROLL = 8;              // work items per thread in flight
+#ifndef GQA_PREP_POS
+#define GQA_PREP_POS 8
+#endif
+#ifndef GQA_PREP_UNROLL
+#define GQA_PREP_UNROLL 8
+#endif
+#ifndef GQA_PREP_MIN_CTAS
+#define GQA_PREP_MIN_CTAS 2
+#endif
+constexpr int PREP_POS = GQA_PREP_POS;          // positions per CTA of the prep kernel
+constexpr int PREP_UNROLL = GQA_PREP_UNROLL;    // work items per thread in flight
 constexpr int PREP_THREADS = 256;
 
 struct Params {
@@ -127,7 +136,7 @@ struct alignas(8) Shared {
 // prep_kernel: for positions [p0, p0+PREP_POS): the cos/sin table, then every Q and K row at those
 // positions rotated into Q' [B*h_q, L, D] and K' [B*h_kv, L, D].
 template <int D>
-__global__ void __launch_bounds__(PREP_THREADS, 2) prep_kernel(const __nv_bfloat16* __restrict__ q,
+__global__ void __launch_bounds__(PREP_THREADS, GQA_PREP_MIN_CTAS) prep_kernel(const __nv_bfloat16* __restrict__ q,
                                                             const __nv_bfloat16* __restrict__ k,
                                                             __nv_bfloat16* __restrict__ qr,
                                                             __nv_bfloat16* __restrict__ kr, int B, int L,

@@ -18,6 +18,7 @@ namespace ptx {
 // Error bits written to the device error word (read back by gqa_last_error()).
 constexpr int kErrBadSeqlen = 1;   // a decode sequence length <= 0 (its output row is zeroed)
 constexpr int kErrTimeout = 2;     // a pipeline wait ran past its limit; the kernel gave up
+constexpr int kErrBadPage = 4;     // a paged decode row had no valid block-table entry (read as zeros)
 
 // Upper bound on any single pipeline wait (nanoseconds of %globaltimer).
 constexpr uint64_t kWaitLimitNs = 1000ull * 1000ull * 1000ull;   // 1 s

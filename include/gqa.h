@@ -47,6 +47,9 @@ extern "C" {
 #define GQA_DEVERR_SEQLEN 1    /* a decode length was <= 0; that sequence's output was zeroed */
 #define GQA_DEVERR_TIMEOUT 2   /* a kernel pipeline wait ran past its limit and gave up;     */
                                /* outputs of that call are undefined                          */
+#define GQA_DEVERR_PAGE 4      /* gqa_decode_paged: a cache row had no valid block-table entry */
+                               /* (page index outside [0, num_pages), or the sequence is longer */
+                               /* than max_pages_per_seq pages); that row was read as zeros     */
 
 /*
  * Causal GQA prefill over whole sequences (page "Qwen2 architecture introduction",
@@ -117,6 +120,27 @@ GQA_API int gqa_set_timing_events(void* start_event, void* stop_event);
  */
 GQA_API int gqa_decode_noalloc(const void* q, const void* kcache, const void* vcache, const int* seqlens,
                                void* out, int B, int h_q, int h_kv, int d, float theta);
+
+/*
+ * gqa_decode_paged -- the decode step of gqa_decode over a paged KV cache (page "从 Qwen 1 到 Qwen 2",
+ * nxmr.cn, §2.4: serving engines such as vLLM keep the cache of each KV head in fixed-size blocks,
+ * PagedAttention).  Same query, positions, softmax and output as gqa_decode; only where cache rows live
+ * differs.
+ *   kpages, vpages [num_pages, page_size, h_kv, d]   un-rotated keys / values; page P slot s holds one
+ *                                                    cache row (all h_kv heads of one position)
+ *   block_table    [B, max_pages_per_seq] int32, DEVICE memory: row j (position j, 0-based) of sequence b
+ *                  lives in page block_table[b][j / page_size], slot j % page_size.  Entries for pages past
+ *                  the end of a sequence are not read.  Pages may be shared between sequences.
+ *   seqlens [B] int32 DEVICE memory, q [B, h_q, d], out [B, h_q, d], d and theta as for gqa_decode.
+ * page_size >= 1 (any value; 16 or a multiple of 16 keeps whole blocks of 16 rows in one page),
+ * num_pages >= 1, max_pages_per_seq >= 1, else GQA_ERR_DIMS.  A table entry outside [0, num_pages), or a
+ * sequence longer than max_pages_per_seq * page_size, is not an API error (the table lives on the
+ * device): the rows concerned are read as zeros, nothing outside kpages / vpages is accessed, and
+ * GQA_DEVERR_PAGE is raised in the device error word.  Workspace and stream as for gqa_decode.
+ */
+GQA_API int gqa_decode_paged(const void* q, const void* kpages, const void* vpages, const int* block_table,
+                             const int* seqlens, void* out, int B, int h_q, int h_kv, int d, int page_size,
+                             int num_pages, int max_pages_per_seq, float theta);
 
 /* Stream for subsequent calls (a cudaStream_t passed as void*; NULL = legacy stream). */
 GQA_API int gqa_set_stream(void* cuda_stream);

@@ -31,6 +31,10 @@ into independent blocks (each block is still the full materialised product):
      p = seqlens[b], attends to all seqlens[b] cached rows (positions
      0 .. p-1).  ``include_self=True`` selects the other reading, where the
      cache already holds the new token and the query sits at p - 1.
+  5. Paged cache (nxmr.cn page, §2.4: PagedAttention keeps the cache of each
+     KV head in fixed-size blocks): the same decode, with position j of
+     sequence b read from slot j % page_size of page block_table[b, j //
+     page_size].  ``decode_paged_ref`` gathers the rows and applies step 4.
 
 Every function is pinned by ``tests/test_oracle_pins.py`` against closed forms,
 invariants the pages state and a brute-force restatement.
@@ -184,6 +188,25 @@ def decode_ref(q, kcache, vcache, seqlens, theta: float, include_self: bool = Fa
     for b in bs:
         o0, o1 = int(off[b]), int(off[b + 1])
         outs.append(decode_one_ref(q[b], kcache[o0:o1], vcache[o0:o1], theta, include_self))
+    return np.stack(outs, axis=0)
+
+
+def decode_paged_ref(q, kpages, vpages, block_table, seqlens, theta: float, batch_rows=None) -> np.ndarray:
+    """Decode step over a paged cache (nxmr.cn page, §2.4: the cache of each KV head kept in blocks).
+
+    kpages/vpages [num_pages, page_size, h_kv, d]; block_table [B, max_pages]: position j of sequence b is
+    slot j % page_size of page block_table[b, j // page_size].  Gathers each sequence's rows in position
+    order and applies the decode definition of decode_one_ref.
+    """
+    kp, vp, bt = np.asarray(kpages), np.asarray(vpages), np.asarray(block_table)
+    page_size = kp.shape[1]
+    seq = [int(x) for x in (seqlens.tolist() if hasattr(seqlens, "tolist") else seqlens)]
+    bs = range(len(seq)) if batch_rows is None else list(batch_rows)
+    outs = []
+    for b in bs:
+        kr = np.stack([kp[bt[b, j // page_size], j % page_size] for j in range(seq[b])])
+        vr = np.stack([vp[bt[b, j // page_size], j % page_size] for j in range(seq[b])])
+        outs.append(decode_one_ref(q[b], kr, vr, theta))
     return np.stack(outs, axis=0)
 
 

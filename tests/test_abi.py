@@ -31,7 +31,7 @@ def codes():
 
 def test_header_declares_the_entry_points():
     names = set(declared())
-    for n in ["gqa_prefill", "gqa_decode", "gqa_set_stream", "gqa_last_error", "gqa_release",
+    for n in ["gqa_prefill", "gqa_decode", "gqa_decode_paged", "gqa_set_stream", "gqa_last_error", "gqa_release",
               "gqa_strerror", "gqa_abi_version", "gqa_set_timing_events"]:
         assert n in names
 
@@ -86,6 +86,31 @@ def test_prefill_validation(lib, args, code):
 ])
 def test_decode_validation(lib, args, code):
     assert lib.gqa_decode(*args) == codes()[code]
+
+
+def paged_args(q=P16, kp=P16, vp=P16, bt=P16, s=P16, out=P16, B=4, h_q=28, h_kv=4, d=128, page=16, npages=64,
+               maxp=8, theta=F):
+    return (q, kp, vp, bt, s, out, B, h_q, h_kv, d, page, npages, maxp, theta)
+
+
+@pytest.mark.parametrize("args,code", [
+    (paged_args(B=-1), "GQA_ERR_DIMS"),
+    (paged_args(page=0), "GQA_ERR_DIMS"),
+    (paged_args(page=-16), "GQA_ERR_DIMS"),
+    (paged_args(npages=0), "GQA_ERR_DIMS"),
+    (paged_args(maxp=0), "GQA_ERR_DIMS"),
+    (paged_args(npages=1 << 30, page=1 << 12), "GQA_ERR_DIMS"),      # storage rows beyond 2^40
+    (paged_args(h_kv=3), "GQA_ERR_DIMS"),
+    (paged_args(d=80), "GQA_ERR_HEAD_DIM"),
+    (paged_args(theta=ctypes.c_float(0.0)), "GQA_ERR_THETA"),
+    (paged_args(bt=None), "GQA_ERR_NULL"),
+    (paged_args(kp=None), "GQA_ERR_NULL"),
+    (paged_args(s=None), "GQA_ERR_NULL"),
+    (paged_args(vp=ctypes.c_void_p(264)), "GQA_ERR_ALIGN"),
+    (paged_args(q=None, kp=None, vp=None, bt=None, s=None, out=None, B=0), "GQA_OK"),
+])
+def test_decode_paged_validation(lib, args, code):
+    assert lib.gqa_decode_paged(*args) == codes()[code]
 
 
 def test_set_stream_accepts_null(lib):
