@@ -378,20 +378,26 @@ def run_ours(args):
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     K, W = args.steps, args.warmup
 
-    def step(evs=None):
+    def step(evs=None, inner=False):
+        """One step; with `inner` the library also records events around its main kernels, which makes
+        the attention launch a plain one (no overlap with the prep kernel), so the headline steps run
+        without them and separate steps time the kernels."""
         flush.zero_()
         if evs:
             evs[0].record()
+        if evs and inner:
             G.set_timing_events(evs[1], evs[2])
         if do_p:
             G.prefill(q, k, v, theta=wp.theta, out=out)
         if evs:
             evs[3].record()
+        if evs and inner:
             G.set_timing_events(evs[4], evs[5])
         if do_d:
             dec_call(qd, s, table)
         if evs:
             evs[6].record()
+        if evs and inner:
             G.set_timing_events(None, None)
 
     for _ in range(W):
@@ -399,7 +405,8 @@ def run_ours(args):
     torch.cuda.synchronize()
     if G.last_error() != 0:
         raise RuntimeError("device error during warm-up")
-    evs = [[ev() for _ in range(7)] for _ in range(K)]
+    evs = [[ev() for _ in range(7)] for _ in range(K)]       # headline steps
+    kevs = [[ev() for _ in range(7)] for _ in range(K)]      # kernel-timing steps
     torch.cuda.synchronize()
 
     barrier()
@@ -409,6 +416,8 @@ def run_ours(args):
         t_wall = time.perf_counter()
         for i in range(K):
             step(evs[i])
+        for i in range(K):
+            step(kevs[i], inner=True)
         torch.cuda.synchronize()
         t_wall = time.perf_counter() - t_wall
     barrier()
@@ -417,9 +426,9 @@ def run_ours(args):
         raise RuntimeError("device error in the timed region")
 
     pre_ms = [e[0].elapsed_time(e[3]) for e in evs]
-    attn_ms = [e[1].elapsed_time(e[2]) if do_p else float("nan") for e in evs]
+    attn_ms = [e[1].elapsed_time(e[2]) if do_p else float("nan") for e in kevs]
     dec_ms = [e[3].elapsed_time(e[6]) for e in evs]
-    split_ms = [e[4].elapsed_time(e[5]) if do_d else float("nan") for e in evs]
+    split_ms = [e[4].elapsed_time(e[5]) if do_d else float("nan") for e in kevs]
     fl = prefill_flops(wp)
     value_tflops = whole_job_rate(fl, 1e-3 * sum(pre_ms) / K, dev) / 1e12   # every rank: same collectives
     pre_mean = reduce_max(sum(pre_ms) / K, dev)
@@ -484,7 +493,9 @@ def run_ours(args):
             "ms_per_step": pre_mean,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic: seeded N(0,1) bf16 Q/K/V and caches drawn on the device; decode lengths U[1,32768]",
-            "config": bench_config(wp, wd),
+            "config": dict(bench_config(wp, wd),
+                           timing=f"{K} headline steps without per-kernel events, then {K} steps with CUDA "
+                                  "events around the attention / split kernels for the roofline"),
             "roofline": {"kernel": "attn_kernel (prefill)", "bound": "tensor", "achieved": achieved_t,
                          "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved_t / peaks["bf16_tflops"],
                          "peak_source": f"{peak_src} bf16 dense (burst)",
@@ -495,7 +506,7 @@ def run_ours(args):
             "e2e": {"value": world * fl / (e2e_pre * 1e-3) / 1e12, "unit": "TFLOP/s",
                     "h2d_bytes_per_step": sum(x.numel() * x.element_size() for x in (q, k, v)),
                     "d2h_bytes_per_step": out.numel() * out.element_size()},
-            "gpu_launches": (2 * do_p + 3 * do_d) * K,
+            "gpu_launches": (2 * do_p + 3 * do_d) * 2 * K,
             "clocks": sampler.summary(),
             "decode": {
                 "workload": wd.desc, "total_cache_rows": total_rows,

@@ -29,6 +29,18 @@ struct DeviceState {
     void* dws = nullptr;          // decode workspace
     size_t dws_bytes = 0;
     void* fixed_scratch = nullptr;   // device address of g_fixed_scratch (gqa_decode_noalloc)
+    bool attn_ready[2] = {false, false};   // attention kernel attributes set and checked (d = 64, 128)
+    // The tensor maps of the last prefill call, reused while every pointer and size matches.
+    struct MapKey {
+        const void *qr, *kr, *v, *out;
+        int B, L, h_q, h_kv, d;
+        bool operator==(const MapKey& o) const {
+            return qr == o.qr && kr == o.kr && v == o.v && out == o.out && B == o.B && L == o.L && h_q == o.h_q &&
+                   h_kv == o.h_kv && d == o.d;
+        }
+    } map_key{};
+    bool maps_valid = false;
+    CUtensorMap maps[4];
 };
 
 DeviceState g_dev[kMaxDevices];
@@ -122,38 +134,26 @@ int check_common(int h_q, int h_kv, int d, float theta) {
     return GQA_OK;
 }
 
+// The four tensor maps of the attention kernel: Q' and K' (3-D, rotated workspace), V and out (4-D, the
+// caller's tensors in place).
 template <int D>
-int launch_prefill(DeviceState* st, const void* q, const void* k, const void* v, void* out, int B, int L, int h_q,
-                   int h_kv, float theta) {
+int encode_prefill_maps(CUtensorMap* maps, const void* qr, const void* kr, const void* v, void* out, int B, int L,
+                        int h_q, int h_kv) {
     using namespace gqa::prefill;
-    // Workspace: Q' [B*h_q, L, D] then K' [B*h_kv, L, D], both bf16, rotated.
-    const size_t qr_bytes = (static_cast<size_t>(B) * h_q * L * D * 2 + 255) & ~size_t(255);
-    const size_t kr_bytes = static_cast<size_t>(B) * h_kv * L * D * 2;
-    if (!ensure(st->ws, st->ws_bytes, qr_bytes + kr_bytes)) return GQA_ERR_ALLOC;
-    auto* qr = static_cast<__nv_bfloat16*>(st->ws);
-    auto* kr = reinterpret_cast<__nv_bfloat16*>(static_cast<uint8_t*>(st->ws) + qr_bytes);
-
-    const int prep_blocks = (L + PREP_POS - 1) / PREP_POS;
-    prep_kernel<D><<<prep_blocks, PREP_THREADS, 0, g_stream>>>(static_cast<const __nv_bfloat16*>(q),
-                                                               static_cast<const __nv_bfloat16*>(k), qr, kr, B, L,
-                                                               h_q, h_kv, std::log2(static_cast<double>(theta)));
-    if (cudaGetLastError() != cudaSuccess) return GQA_ERR_LAUNCH;
-    // (the host work below overlaps the prep kernel)
-
     if (!get_encoder()) return GQA_ERR_LAUNCH;
-    CUtensorMap tm_q, tm_k, tm_v, tm_o;
+    CUtensorMap &tm_q = maps[0], &tm_k = maps[1], &tm_v = maps[2], &tm_o = maps[3];
     const cuuint32_t box3[3] = {64, BM, 1};
     {   // Q' [B*h_q, L, D]
         const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(L),
                                     static_cast<cuuint64_t>(B) * h_q};
         const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(L) * D * 2};
-        if (!encode_bf16(&tm_q, qr, 3, dims, strides, box3)) return GQA_ERR_LAUNCH;
+        if (!encode_bf16(&tm_q, const_cast<void*>(qr), 3, dims, strides, box3)) return GQA_ERR_LAUNCH;
     }
     {   // K' [B*h_kv, L, D]
         const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(L),
                                     static_cast<cuuint64_t>(B) * h_kv};
         const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(L) * D * 2};
-        if (!encode_bf16(&tm_k, kr, 3, dims, strides, box3)) return GQA_ERR_LAUNCH;
+        if (!encode_bf16(&tm_k, const_cast<void*>(kr), 3, dims, strides, box3)) return GQA_ERR_LAUNCH;
     }
     const cuuint32_t box4[4] = {64, 1, BN, 1};
     {   // V [B, L, h_kv, D], read in place
@@ -172,6 +172,36 @@ int launch_prefill(DeviceState* st, const void* q, const void* k, const void* v,
         if (!encode_bf16(&tm_o, out, 4, dims, strides, box_o)) return GQA_ERR_LAUNCH;
     }
 
+    return GQA_OK;
+}
+
+template <int D>
+int launch_prefill(DeviceState* st, const void* q, const void* k, const void* v, void* out, int B, int L, int h_q,
+                   int h_kv, float theta) {
+    using namespace gqa::prefill;
+    // Workspace: Q' [B*h_q, L, D] then K' [B*h_kv, L, D], both bf16, rotated.
+    const size_t qr_bytes = (static_cast<size_t>(B) * h_q * L * D * 2 + 255) & ~size_t(255);
+    const size_t kr_bytes = static_cast<size_t>(B) * h_kv * L * D * 2;
+    if (!ensure(st->ws, st->ws_bytes, qr_bytes + kr_bytes)) return GQA_ERR_ALLOC;
+    auto* qr = static_cast<__nv_bfloat16*>(st->ws);
+    auto* kr = reinterpret_cast<__nv_bfloat16*>(static_cast<uint8_t*>(st->ws) + qr_bytes);
+
+    const int prep_blocks = (L + PREP_POS - 1) / PREP_POS;
+    prep_kernel<D><<<prep_blocks, PREP_THREADS, 0, g_stream>>>(static_cast<const __nv_bfloat16*>(q),
+                                                               static_cast<const __nv_bfloat16*>(k), qr, kr, B, L,
+                                                               h_q, h_kv, std::log2(static_cast<double>(theta)));
+    if (cudaGetLastError() != cudaSuccess) return GQA_ERR_LAUNCH;
+    // (the host work below overlaps the prep kernel)
+
+    const DeviceState::MapKey key{qr, kr, v, out, B, L, h_q, h_kv, D};
+    if (!st->maps_valid || !(st->map_key == key)) {
+        st->maps_valid = false;
+        const int rc = encode_prefill_maps<D>(st->maps, qr, kr, v, out, B, L, h_q, h_kv);
+        if (rc != GQA_OK) return rc;
+        st->map_key = key;
+        st->maps_valid = true;
+    }
+
     Params p;
     p.out = static_cast<__nv_bfloat16*>(out);
     p.B = B;
@@ -188,16 +218,35 @@ int launch_prefill(DeviceState* st, const void* q, const void* k, const void* v,
     p.total_work = static_cast<int>(total);
     // Persistent: one CTA per SM (each holds a whole SM's tensor memory), at most one per work item.
     const int grid = static_cast<int>(total < st->num_sms ? total : st->num_sms);
-    if (cudaFuncSetAttribute(attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, Layout<D>::DYN) !=
+    bool& ready = st->attn_ready[D == 128 ? 1 : 0];
+    if (!ready) {
+        if (cudaFuncSetAttribute(attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, Layout<D>::DYN) !=
+            cudaSuccess)
+            return GQA_ERR_LAUNCH;
+        // The in-kernel register split (setmaxnreg) is only valid for this exact launch budget.
+        cudaFuncAttributes fa;
+        if (cudaFuncGetAttributes(&fa, attn_kernel<D>) != cudaSuccess || fa.numRegs != LAUNCH_REGS)
+            return GQA_ERR_LAUNCH;
+        ready = true;
+    }
+    // Programmatic dependent launch: the attention CTAs may start (barrier set-up, tensor-memory
+    // allocation) while the prep kernel drains, and wait for its results with griddepcontrol.wait.
+    // With timing events the start event sits between the two kernels, so the launch is plain.
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(NUM_THREADS);
+    cfg.dynamicSmemBytes = Layout<D>::DYN;
+    cfg.stream = g_stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    const bool timed = g_ev_start && g_ev_stop;
+    cfg.attrs = attr;
+    cfg.numAttrs = timed ? 0 : 1;
+    mark(g_ev_start);
+    if (cudaLaunchKernelEx(&cfg, attn_kernel<D>, st->maps[0], st->maps[1], st->maps[2], st->maps[3], p) !=
         cudaSuccess)
         return GQA_ERR_LAUNCH;
-    // The in-kernel register split (setmaxnreg) is only valid for this exact launch budget.
-    cudaFuncAttributes fa;
-    if (cudaFuncGetAttributes(&fa, attn_kernel<D>) != cudaSuccess || fa.numRegs != LAUNCH_REGS)
-        return GQA_ERR_LAUNCH;
-    mark(g_ev_start);
-    attn_kernel<D><<<grid, NUM_THREADS, Layout<D>::DYN, g_stream>>>(tm_q, tm_k, tm_v, tm_o, p);
-    if (cudaGetLastError() != cudaSuccess) return GQA_ERR_LAUNCH;
     mark(g_ev_stop);
     return GQA_OK;
 }
@@ -451,6 +500,7 @@ void gqa_release(void) {
         if (st.ws) cudaFree(st.ws);
         if (st.dws) cudaFree(st.dws);
         st.ws = st.dws = nullptr;
+        st.maps_valid = false;
         st.ws_bytes = st.dws_bytes = 0;
     }
     cudaSetDevice(cur);

@@ -147,6 +147,9 @@ __global__ void __launch_bounds__(PREP_THREADS, GQA_PREP_MIN_CTAS) prep_kernel(c
     // the 8 chunks of a row (read by 8 neighbouring lanes) fall in 8 different shared-memory banks.
     constexpr int TROW = H + H / 8;
     __shared__ float2 tab[PREP_POS * TROW];
+    // The attention kernel launched after this one may be scheduled now; it waits for this grid's
+    // results (griddepcontrol.wait) before reading Q' or K'.
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     __shared__ double finv[H];
     const int p0 = blockIdx.x * PREP_POS;
     const int heads = h_q + h_kv;
@@ -342,6 +345,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    // Q' and K' come from the prep kernel just before this one (programmatic dependent launch): wait for
+    // that grid to complete and its writes to be visible.  A no-op for a plain launch.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const uint32_t tmem = sh.tmem_base;
     volatile int* abort = &sh.abort;
 
