@@ -91,6 +91,35 @@ def prefill_inputs(w: Workload, device: str = "cpu"):
     return q, k, v
 
 
+# Hidden size of the Qwen2 models whose head shapes the workloads use (Qwen2-0.5B: 896, Qwen2-7B: 3584,
+# Qwen2-72B: 8192): the K dimension of the fused QKV projection.
+D_MODEL = {(14, 2, 64): 896, (28, 4, 128): 3584, (64, 8, 128): 8192}
+
+
+def qkv_inputs(w: Workload, d_model: int | None = None, device: str = "cpu", bias: bool = True):
+    """Synthetic inputs of the fused QKV projection for the prefill workload w.
+
+    x [B, L, d_model] ~ N(0, 1) (hidden states after RMSNorm); w_qkv [(h_q + 2 h_kv) d, d_model]
+    ~ N(0, 1/d_model), the rows of W_Q^T, W_K^T, W_V^T stacked (the nn.Linear weight layout);
+    b_qkv [(h_q + 2 h_kv) d] ~ N(0, 0.1^2) or None.  All bf16.  The weight scale keeps projected values
+    near unit size, as in trained models.
+    """
+    assert w.kind == "prefill"
+    dm = d_model or D_MODEL[(w.h_q, w.h_kv, w.d)]
+    n = (w.h_q + 2 * w.h_kv) * w.d
+    gen = _gen(w.seed + 31337, device)
+    x = _randn_bf16((w.B * w.L, dm), gen, device).view(w.B, w.L, dm)
+    wq = torch.empty((n, dm), dtype=torch.bfloat16, device=device)
+    for s0 in range(0, n, 1024):
+        e = min(n, s0 + 1024)
+        wq[s0:e] = (torch.randn((e - s0, dm), generator=gen, dtype=torch.float32, device=device)
+                    / (dm ** 0.5)).to(torch.bfloat16)
+    b = None
+    if bias:
+        b = (0.1 * torch.randn((n,), generator=gen, dtype=torch.float32, device=device)).to(torch.bfloat16)
+    return x, wq, b
+
+
 def decode_inputs(w: Workload, device: str = "cpu", seqlens=None):
     """seqlens int32 [B]; q [B,h_q,d]; kcache, vcache packed [sum(seqlens), h_kv, d].
 

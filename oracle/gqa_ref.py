@@ -35,6 +35,10 @@ into independent blocks (each block is still the full materialised product):
      KV head in fixed-size blocks): the same decode, with position j of
      sequence b read from slot j % page_size of page block_table[b, j //
      page_size].  ``decode_paged_ref`` gathers the rows and applies step 4.
+  6. QKV projection (aicoding.csdn.net page, §4.1.3 steps 1-3): Q, K, V are
+     the hidden states times W_Q, W_K, W_V plus the bias, split into h_q and
+     h_kv heads; Q and K are then rotated as in step 1.
+     ``qkv_rope_ref`` writes it out with one matrix product.
 
 Every function is pinned by ``tests/test_oracle_pins.py`` against closed forms,
 invariants the pages state and a brute-force restatement.
@@ -208,6 +212,34 @@ def decode_paged_ref(q, kpages, vpages, block_table, seqlens, theta: float, batc
         vr = np.stack([vp[bt[b, j // page_size], j % page_size] for j in range(seq[b])])
         outs.append(decode_one_ref(q[b], kr, vr, theta))
     return np.stack(outs, axis=0)
+
+
+def qkv_rope_ref(x, w_qkv, b_qkv, h_q: int, h_kv: int, d: int, theta: float):
+    """Steps 1-3 of the aicoding.csdn.net page, §4.1.3: projections with bias, split into heads, RoPE.
+
+    x [B, L, d_model]; w_qkv [(h_q + 2 h_kv) d, d_model] holds the rows of W_Q^T, W_K^T, W_V^T (so the
+    projection is x @ w_qkv^T, i.e. X W with W = w_qkv^T); b_qkv [(h_q + 2 h_kv) d] or None.  Positions
+    are 0 .. L-1 in every batch row.  Returns float64 arrays in the layouts the CUDA path writes:
+    qr [B, h_q, L, d] and kr [B, h_kv, L, d] rotated (head-major), k and v [B, L, h_kv, d] un-rotated
+    (token-major: the packed cache rows of the sequence).
+    """
+    xf, wf = as_f64(x), as_f64(w_qkv)
+    B, L, _ = xf.shape
+    y = xf @ wf.T                                         # [B, L, (h_q + 2 h_kv) d]
+    if b_qkv is not None:
+        y = y + as_f64(b_qkv)[None, None, :]
+    q = y[..., :h_q * d].reshape(B, L, h_q, d)
+    k = y[..., h_q * d:(h_q + h_kv) * d].reshape(B, L, h_kv, d)
+    v = y[..., (h_q + h_kv) * d:].reshape(B, L, h_kv, d)
+    pos = np.arange(L)
+    qr = np.stack([rope(q[b], pos, theta) for b in range(B)]).transpose(0, 2, 1, 3)
+    kr = np.stack([rope(k[b], pos, theta) for b in range(B)]).transpose(0, 2, 1, 3)
+    return qr, kr, k, v
+
+
+def qkv_flops(B: int, L: int, d_model: int, h_q: int, h_kv: int, d: int) -> float:
+    """FLOP count of the fused projection: one GEMM of [B*L, d_model] x [d_model, (h_q + 2 h_kv) d]."""
+    return 2.0 * B * L * d_model * (h_q + 2 * h_kv) * d
 
 
 def prefill_flops(B: int, L: int, h_q: int, d: int) -> float:
