@@ -45,6 +45,10 @@ def load() -> ctypes.CDLL:
     lib.gqa_decode.restype = i
     lib.gqa_decode_paged.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, f]
     lib.gqa_decode_paged.restype = i
+    lib.gqa_qkv_rope.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f]
+    lib.gqa_qkv_rope.restype = i
+    lib.gqa_prefill_rotated.argtypes = [vp, vp, vp, vp, i, i, i, i, i]
+    lib.gqa_prefill_rotated.restype = i
     lib.gqa_set_timing_events.argtypes = [vp, vp]
     lib.gqa_set_timing_events.restype = i
     lib.gqa_set_stream.argtypes = [vp]
@@ -159,6 +163,59 @@ def decode_paged(q: torch.Tensor, kpages: torch.Tensor, vpages: torch.Tensor, bl
                                      float(theta))
     if rc != GQA_OK:
         raise GQAError(rc, "gqa_decode_paged")
+    return out
+
+
+def qkv_rope(x: torch.Tensor, w_qkv: torch.Tensor, b_qkv: torch.Tensor | None, h_q: int, h_kv: int,
+             theta: float = 1.0e6, out=None):
+    """Fused QKV projection + bias + RoPE.  x [B, L, d_model]; w_qkv [(h_q + 2 h_kv) d, d_model] (nn.Linear
+    layout); b_qkv [(h_q + 2 h_kv) d] or None.  Returns (qr [B,h_q,L,d], kr [B,h_kv,L,d] rotated,
+    k [B,L,h_kv,d] raw, v [B,L,h_kv,d]); `out` may give those four tensors (e.g. k, v inside a cache)."""
+    if x.dim() != 3 or w_qkv.dim() != 2:
+        raise ValueError("x must be [B, L, d_model] and w_qkv [(h_q + 2 h_kv) d, d_model]")
+    B, L, dm = x.shape
+    n = w_qkv.shape[0]
+    if n % (h_q + 2 * h_kv) != 0:
+        raise ValueError(f"w_qkv has {n} rows, not a multiple of h_q + 2 h_kv = {h_q + 2 * h_kv}")
+    d = n // (h_q + 2 * h_kv)
+    _check(x, "x", None)
+    _check(w_qkv, "w_qkv", (n, dm))
+    if b_qkv is not None:
+        _check(b_qkv, "b_qkv", (n,))
+    if out is None:
+        out = (x.new_empty(B, h_q, L, d), x.new_empty(B, h_kv, L, d), x.new_empty(B, L, h_kv, d),
+               x.new_empty(B, L, h_kv, d))
+    qr, kr, k, v = out
+    _check(qr, "qr", (B, h_q, L, d))
+    _check(kr, "kr", (B, h_kv, L, d))
+    _check(k, "k", (B, L, h_kv, d))
+    _check(v, "v", (B, L, h_kv, d))
+    with torch.cuda.device(x.device):
+        _stream(x.device)
+        rc = load().gqa_qkv_rope(_ptr(x), _ptr(w_qkv), _ptr(b_qkv), _ptr(qr), _ptr(kr), _ptr(k), _ptr(v),
+                                 B, L, dm, h_q, h_kv, d, float(theta))
+    if rc != GQA_OK:
+        raise GQAError(rc, "gqa_qkv_rope")
+    return qr, kr, k, v
+
+
+def prefill_rotated(qr: torch.Tensor, kr: torch.Tensor, v: torch.Tensor, out: torch.Tensor | None = None):
+    """Causal GQA attention on rotated inputs: qr [B,h_q,L,d], kr [B,h_kv,L,d], v [B,L,h_kv,d] -> [B,L,h_q,d]."""
+    if qr.dim() != 4 or kr.dim() != 4 or v.dim() != 4:
+        raise ValueError("qr, kr and v must be 4-D")
+    B, h_q, L, d = qr.shape
+    h_kv = kr.shape[1]
+    _check(qr, "qr", None)
+    _check(kr, "kr", (B, h_kv, L, d))
+    _check(v, "v", (B, L, h_kv, d))
+    if out is None:
+        out = qr.new_empty(B, L, h_q, d)
+    _check(out, "out", (B, L, h_q, d))
+    with torch.cuda.device(qr.device):
+        _stream(qr.device)
+        rc = load().gqa_prefill_rotated(_ptr(qr), _ptr(kr), _ptr(v), _ptr(out), B, L, h_q, h_kv, d)
+    if rc != GQA_OK:
+        raise GQAError(rc, "gqa_prefill_rotated")
     return out
 
 

@@ -11,6 +11,7 @@
 #include "../../include/gqa.h"
 #include "decode_sm100.cuh"
 #include "prefill_sm100.cuh"
+#include "qkv_sm100.cuh"
 
 namespace {
 
@@ -41,6 +42,15 @@ struct DeviceState {
     } map_key{};
     bool maps_valid = false;
     CUtensorMap maps[4];
+    // QKV projection: the cos / sin table of the last (L, d, theta), and the last pair of tensor maps.
+    void* tab = nullptr;
+    size_t tab_bytes = 0;
+    int tab_L = -1, tab_d = 0;
+    float tab_theta = 0.f;
+    bool qkv_ready[2] = {false, false};
+    const void* qkv_key[2] = {nullptr, nullptr};
+    long long qkv_dims[3] = {0, 0, 0};
+    CUtensorMap qkv_maps[2];
 };
 
 DeviceState g_dev[kMaxDevices];
@@ -175,24 +185,13 @@ int encode_prefill_maps(CUtensorMap* maps, const void* qr, const void* kr, const
     return GQA_OK;
 }
 
+// The attention kernel over rotated Q' [B, h_q, L, D], K' [B, h_kv, L, D] and V [B, L, h_kv, D].  With
+// `dependent`, it is launched as a programmatic dependent of the kernel just before it on the stream
+// (the prep or projection kernel that writes Q' and K').
 template <int D>
-int launch_prefill(DeviceState* st, const void* q, const void* k, const void* v, void* out, int B, int L, int h_q,
-                   int h_kv, float theta) {
+int launch_attention(DeviceState* st, const void* qr, const void* kr, const void* v, void* out, int B, int L,
+                     int h_q, int h_kv, bool dependent) {
     using namespace gqa::prefill;
-    // Workspace: Q' [B*h_q, L, D] then K' [B*h_kv, L, D], both bf16, rotated.
-    const size_t qr_bytes = (static_cast<size_t>(B) * h_q * L * D * 2 + 255) & ~size_t(255);
-    const size_t kr_bytes = static_cast<size_t>(B) * h_kv * L * D * 2;
-    if (!ensure(st->ws, st->ws_bytes, qr_bytes + kr_bytes)) return GQA_ERR_ALLOC;
-    auto* qr = static_cast<__nv_bfloat16*>(st->ws);
-    auto* kr = reinterpret_cast<__nv_bfloat16*>(static_cast<uint8_t*>(st->ws) + qr_bytes);
-
-    const int prep_blocks = (L + PREP_POS - 1) / PREP_POS;
-    prep_kernel<D><<<prep_blocks, PREP_THREADS, 0, g_stream>>>(static_cast<const __nv_bfloat16*>(q),
-                                                               static_cast<const __nv_bfloat16*>(k), qr, kr, B, L,
-                                                               h_q, h_kv, std::log2(static_cast<double>(theta)));
-    if (cudaGetLastError() != cudaSuccess) return GQA_ERR_LAUNCH;
-    // (the host work below overlaps the prep kernel)
-
     const DeviceState::MapKey key{qr, kr, v, out, B, L, h_q, h_kv, D};
     if (!st->maps_valid || !(st->map_key == key)) {
         st->maps_valid = false;
@@ -230,7 +229,7 @@ int launch_prefill(DeviceState* st, const void* q, const void* k, const void* v,
         ready = true;
     }
     // Programmatic dependent launch: the attention CTAs may start (barrier set-up, tensor-memory
-    // allocation) while the prep kernel drains, and wait for its results with griddepcontrol.wait.
+    // allocation) while the previous kernel drains, and wait for its results with griddepcontrol.wait.
     // With timing events the start event sits between the two kernels, so the launch is plain.
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
@@ -242,11 +241,104 @@ int launch_prefill(DeviceState* st, const void* q, const void* k, const void* v,
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     const bool timed = g_ev_start && g_ev_stop;
     cfg.attrs = attr;
-    cfg.numAttrs = timed ? 0 : 1;
+    cfg.numAttrs = (dependent && !timed) ? 1 : 0;
     mark(g_ev_start);
     if (cudaLaunchKernelEx(&cfg, attn_kernel<D>, st->maps[0], st->maps[1], st->maps[2], st->maps[3], p) !=
         cudaSuccess)
         return GQA_ERR_LAUNCH;
+    mark(g_ev_stop);
+    return GQA_OK;
+}
+
+template <int D>
+int launch_prefill(DeviceState* st, const void* q, const void* k, const void* v, void* out, int B, int L, int h_q,
+                   int h_kv, float theta) {
+    using namespace gqa::prefill;
+    // Workspace: Q' [B*h_q, L, D] then K' [B*h_kv, L, D], both bf16, rotated.
+    const size_t qr_bytes = (static_cast<size_t>(B) * h_q * L * D * 2 + 255) & ~size_t(255);
+    const size_t kr_bytes = static_cast<size_t>(B) * h_kv * L * D * 2;
+    if (!ensure(st->ws, st->ws_bytes, qr_bytes + kr_bytes)) return GQA_ERR_ALLOC;
+    auto* qr = static_cast<__nv_bfloat16*>(st->ws);
+    auto* kr = reinterpret_cast<__nv_bfloat16*>(static_cast<uint8_t*>(st->ws) + qr_bytes);
+
+    const int prep_blocks = (L + PREP_POS - 1) / PREP_POS;
+    prep_kernel<D><<<prep_blocks, PREP_THREADS, 0, g_stream>>>(static_cast<const __nv_bfloat16*>(q),
+                                                               static_cast<const __nv_bfloat16*>(k), qr, kr, B, L,
+                                                               h_q, h_kv, std::log2(static_cast<double>(theta)));
+    if (cudaGetLastError() != cudaSuccess) return GQA_ERR_LAUNCH;
+    return launch_attention<D>(st, qr, kr, v, out, B, L, h_q, h_kv, true);
+}
+
+// The cos / sin table for positions 0 .. L-1, rebuilt only when (L, d, theta) changes.
+template <int D>
+int ensure_rope_table(DeviceState* st, int L, float theta) {
+    using namespace gqa::qkv;
+    if (st->tab && st->tab_L >= L && st->tab_d == D && st->tab_theta == theta) return GQA_OK;
+    const size_t bytes = static_cast<size_t>(L) * (D / 2) * sizeof(float2);
+    if (!ensure(st->tab, st->tab_bytes, bytes)) return GQA_ERR_ALLOC;
+    const long long n = static_cast<long long>(L) * (D / 2);
+    rope_table_kernel<D><<<static_cast<unsigned>((n + TABLE_THREADS - 1) / TABLE_THREADS), TABLE_THREADS, 0,
+                           g_stream>>>(static_cast<float2*>(st->tab), L, std::log2(static_cast<double>(theta)));
+    if (cudaGetLastError() != cudaSuccess) return GQA_ERR_LAUNCH;
+    st->tab_L = L;
+    st->tab_d = D;
+    st->tab_theta = theta;
+    return GQA_OK;
+}
+
+template <int D>
+int launch_qkv(DeviceState* st, const void* x, const void* w, const void* bias, void* qr, void* kr, void* k,
+               void* v, int B, int L, int d_model, int h_q, int h_kv, float theta) {
+    using namespace gqa::qkv;
+    int rc = ensure_rope_table<D>(st, L, theta);
+    if (rc != GQA_OK) return rc;
+    const long long T = static_cast<long long>(B) * L;
+    const int N = (h_q + 2 * h_kv) * D;
+    if (!get_encoder()) return GQA_ERR_LAUNCH;
+    if (st->qkv_key[0] != x || st->qkv_key[1] != w || st->qkv_dims[0] != T || st->qkv_dims[1] != N ||
+        st->qkv_dims[2] != d_model) {
+        st->qkv_key[0] = st->qkv_key[1] = nullptr;
+        const cuuint64_t dx[2] = {static_cast<cuuint64_t>(d_model), static_cast<cuuint64_t>(T)};
+        const cuuint64_t sx[1] = {static_cast<cuuint64_t>(d_model) * 2};
+        const cuuint32_t bx[2] = {BK, BM};
+        if (!encode_bf16(&st->qkv_maps[0], const_cast<void*>(x), 2, dx, sx, bx)) return GQA_ERR_LAUNCH;
+        const cuuint64_t dw[2] = {static_cast<cuuint64_t>(d_model), static_cast<cuuint64_t>(N)};
+        const cuuint32_t bw[2] = {BK, BN};
+        if (!encode_bf16(&st->qkv_maps[1], const_cast<void*>(w), 2, dw, sx, bw)) return GQA_ERR_LAUNCH;
+        st->qkv_key[0] = x;
+        st->qkv_key[1] = w;
+        st->qkv_dims[0] = T;
+        st->qkv_dims[1] = N;
+        st->qkv_dims[2] = d_model;
+    }
+    Params p;
+    p.bias = static_cast<const __nv_bfloat16*>(bias);
+    p.tab = static_cast<const float2*>(st->tab);
+    p.qr = static_cast<__nv_bfloat16*>(qr);
+    p.kr = static_cast<__nv_bfloat16*>(kr);
+    p.k = static_cast<__nv_bfloat16*>(k);
+    p.v = static_cast<__nv_bfloat16*>(v);
+    p.T = static_cast<int>(T);
+    p.L = L;
+    p.N = N;
+    p.h_q = h_q;
+    p.h_kv = h_kv;
+    p.n_ntiles = (N + BN - 1) / BN;
+    const long long mtiles = (T + BM - 1) / BM;
+    if (mtiles * p.n_ntiles > 0x7fffffffLL) return GQA_ERR_DIMS;
+    p.n_tiles = static_cast<int>(mtiles * p.n_ntiles);
+    p.kblocks = (d_model + BK - 1) / BK;
+    p.err = st->err;
+    bool& ready = st->qkv_ready[D == 128 ? 1 : 0];
+    if (!ready) {
+        if (cudaFuncSetAttribute(qkv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, DYN) != cudaSuccess)
+            return GQA_ERR_LAUNCH;
+        ready = true;
+    }
+    const int grid = p.n_tiles < st->num_sms ? p.n_tiles : st->num_sms;
+    mark(g_ev_start);
+    qkv_kernel<D><<<grid, NUM_THREADS, DYN, g_stream>>>(st->qkv_maps[0], st->qkv_maps[1], p);
+    if (cudaGetLastError() != cudaSuccess) return GQA_ERR_LAUNCH;
     mark(g_ev_stop);
     return GQA_OK;
 }
@@ -477,6 +569,41 @@ int gqa_decode_paged(const void* q, const void* kpages, const void* vpages, cons
                                         page_size, num_pages, max_pages_per_seq);
 }
 
+int gqa_qkv_rope(const void* x, const void* w_qkv, const void* b_qkv, void* qr, void* kr, void* k, void* v, int B,
+                 int L, int d_model, int h_q, int h_kv, int d, float theta) {
+    if (B < 0 || L < 0 || d_model <= 0 || d_model % 8 != 0) return GQA_ERR_DIMS;
+    int rc = check_common(h_q, h_kv, d, theta);
+    if (rc != GQA_OK) return rc;
+    if (B == 0 || L == 0) return GQA_OK;
+    if (!x || !w_qkv || !qr || !kr || !k || !v) return GQA_ERR_NULL;
+    if (!aligned16(x) || !aligned16(w_qkv) || !aligned16(qr) || !aligned16(kr) || !aligned16(k) || !aligned16(v) ||
+        (b_qkv && !aligned16(b_qkv)))
+        return GQA_ERR_ALIGN;
+    // Token rows and output columns are TMA coordinates (32-bit); positions stay below 2^30.
+    if (static_cast<long long>(B) * L > 0x7fffffffLL || L > (1 << 30) ||
+        static_cast<long long>(h_q + 2 * h_kv) * d > 0x7fffffffLL)
+        return GQA_ERR_DIMS;
+    DeviceState* st = device_state(&rc);
+    if (!st) return rc;
+    return d == 64 ? launch_qkv<64>(st, x, w_qkv, b_qkv, qr, kr, k, v, B, L, d_model, h_q, h_kv, theta)
+                   : launch_qkv<128>(st, x, w_qkv, b_qkv, qr, kr, k, v, B, L, d_model, h_q, h_kv, theta);
+}
+
+int gqa_prefill_rotated(const void* qr, const void* kr, const void* v, void* out, int B, int L, int h_q, int h_kv,
+                        int d) {
+    if (B < 0 || L < 0) return GQA_ERR_DIMS;
+    int rc = check_common(h_q, h_kv, d, 1.0f);
+    if (rc != GQA_OK) return rc;
+    if (B == 0 || L == 0) return GQA_OK;
+    if (!qr || !kr || !v || !out) return GQA_ERR_NULL;
+    if (!aligned16(qr) || !aligned16(kr) || !aligned16(v) || !aligned16(out)) return GQA_ERR_ALIGN;
+    if (static_cast<long long>(B) * (h_q + h_kv) * 64 > 0x7fffffffLL || L > (1 << 30)) return GQA_ERR_DIMS;
+    DeviceState* st = device_state(&rc);
+    if (!st) return rc;
+    return d == 64 ? launch_attention<64>(st, qr, kr, v, out, B, L, h_q, h_kv, true)
+                   : launch_attention<128>(st, qr, kr, v, out, B, L, h_q, h_kv, true);
+}
+
 int gqa_last_error(void) {
     int rc = GQA_OK;
     DeviceState* st = device_state(&rc);
@@ -494,11 +621,15 @@ void gqa_release(void) {
     if (cudaGetDevice(&cur) != cudaSuccess) return;
     for (int dev = 0; dev < kMaxDevices; ++dev) {
         DeviceState& st = g_dev[dev];
-        if (!st.ws && !st.dws) continue;
+        if (!st.ws && !st.dws && !st.tab) continue;
         cudaSetDevice(dev);
         cudaDeviceSynchronize();
         if (st.ws) cudaFree(st.ws);
         if (st.dws) cudaFree(st.dws);
+        if (st.tab) cudaFree(st.tab);
+        st.tab = nullptr;
+        st.tab_bytes = 0;
+        st.tab_L = -1;
         st.ws = st.dws = nullptr;
         st.maps_valid = false;
         st.ws_bytes = st.dws_bytes = 0;

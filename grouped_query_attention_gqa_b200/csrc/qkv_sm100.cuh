@@ -1,0 +1,273 @@
+// Fused QKV projection + bias + RoPE on sm_100a (page "Qwen2 architecture introduction",
+// aicoding.csdn.net, §4.1.3 steps 1-3): Y = X W^T + b for the stacked weight W = [W_Q^T; W_K^T; W_V^T]
+// ([(h_q + 2 h_kv) d, d_model], the nn.Linear layout), split into heads; Q and K heads are rotated at
+// their positions.  One pass writes everything the attention step and the KV cache need:
+//   qr [B, h_q,  L, d]  rotated Q, head-major (the attention kernel's Q' layout)
+//   kr [B, h_kv, L, d]  rotated K, head-major (its K' layout)
+//   k  [B, L, h_kv, d]  raw K, token-major: the packed cache rows of the sequences, back to back
+//   v  [B, L, h_kv, d]  V, token-major (cache rows; the attention kernel reads V in this layout)
+//
+// qkv_kernel is a persistent tcgen05 GEMM, one CTA per SM, over 128 x 256 output tiles (128 tokens,
+// 256 output columns = 2 heads of d = 128 or 4 of d = 64):
+//   warp 0     TMA producer: 64-wide K blocks of X (128 x 64) and W (256 x 64) into a 4-stage ring
+//   warp 1     MMA issuer: 4 x tcgen05.mma M128 N256 K16 per K block into one of two TMEM accumulators
+//   warps 2-5  epilogue: one TMEM lane (token row) per thread; per head: + bias, rotate, round, store
+// The two accumulators (2 x 256 TMEM columns) let the epilogue of one tile overlap the main loop of the
+// next.  cos / sin come from a per-position table built once per (L, d, theta).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cstdint>
+
+#include "rope.cuh"
+#include "sm100_ptx.cuh"
+
+namespace gqa {
+namespace qkv {
+
+using namespace ptx;
+
+constexpr int BM = 128;                  // tokens per tile (MMA M, TMEM lanes)
+constexpr int BN = 256;                  // output columns per tile (MMA N)
+constexpr int BK = 64;                   // K block: one 128-byte swizzle atom of bf16
+constexpr int STAGES = 4;
+constexpr int NUM_THREADS = 192;
+constexpr int WARP_TMA = 0, WARP_MMA = 1;
+constexpr int A_BYTES = BM * BK * 2;     // 16 KB
+constexpr int B_BYTES = BN * BK * 2;     // 32 KB
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int DYN = STAGES * STAGE_BYTES + 1024;
+constexpr int TMEM_COLS = 2 * BN;
+constexpr int TABLE_THREADS = 256;
+
+struct Params {
+    const __nv_bfloat16* bias;   // [N] or nullptr
+    const float2* tab;           // [L, d/2] (cos, sin) of pos * theta^(-2i/d)
+    __nv_bfloat16* qr;
+    __nv_bfloat16* kr;
+    __nv_bfloat16* k;
+    __nv_bfloat16* v;
+    int T, L, N, h_q, h_kv;
+    int n_ntiles, n_tiles, kblocks;
+    int* err;
+};
+
+struct alignas(8) Shared {
+    uint64_t full[STAGES], empty[STAGES];
+    uint64_t acc_full[2], acc_empty[2];
+    uint64_t mma_done;
+    uint32_t tmem_base;
+    int abort;
+};
+
+// ---------------------------------------------------------------------------------------------
+// The cos / sin table: tab[pos * d/2 + i] = (cos, sin)(pos * theta^(-2i/d)), the angle formed in double
+// precision (rope_cossin).
+template <int D>
+__global__ void __launch_bounds__(TABLE_THREADS) rope_table_kernel(float2* __restrict__ tab, int L,
+                                                                   double log2_theta) {
+    constexpr int H = D / 2;
+    const int64_t e = static_cast<int64_t>(blockIdx.x) * TABLE_THREADS + threadIdx.x;
+    if (e >= static_cast<int64_t>(L) * H) return;
+    const int pos = static_cast<int>(e / H), i = static_cast<int>(e % H);
+    float c, s;
+    rope_cossin(static_cast<double>(pos), exp2(-(2.0 * i / D) * log2_theta), c, s);
+    tab[e] = make_float2(c, s);
+}
+
+// ---------------------------------------------------------------------------------------------
+// One head (D columns starting at n0) of one token row, in place: + bias, rotate if Q or K, round, store.
+template <int D>
+__device__ __forceinline__ void store_head(const Params& p, float (&y)[D], int n0, int b, int pos) {
+    constexpr int H = D / 2;
+    if (p.bias) {
+        const uint4* bb = reinterpret_cast<const uint4*>(p.bias + n0);
+#pragma unroll
+        for (int c = 0; c < D / 8; ++c) {
+            const uint4 w = bb[c];
+            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                y[8 * c + 2 * e] += bf16lo_to_f32(ws[e]);
+                y[8 * c + 2 * e + 1] += bf16hi_to_f32(ws[e]);
+            }
+        }
+    }
+    const int head = n0 / D;
+    auto store_row = [&](__nv_bfloat16* dst, const float* z) {
+        uint4* o = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+        for (int c = 0; c < D / 8; ++c)
+            o[c] = make_uint4(pack_bf16x2(z[8 * c], z[8 * c + 1]), pack_bf16x2(z[8 * c + 2], z[8 * c + 3]),
+                              pack_bf16x2(z[8 * c + 4], z[8 * c + 5]), pack_bf16x2(z[8 * c + 6], z[8 * c + 7]));
+    };
+    auto rotate = [&](float* z) {
+        const float4* t = reinterpret_cast<const float4*>(p.tab + static_cast<int64_t>(pos) * H);
+#pragma unroll
+        for (int c = 0; c < H / 2; ++c) {
+            const float4 cs = t[c];   // (cos, sin) of frequencies 2c and 2c + 1
+            float a0, b0, a1, b1;
+            rope_rotate(z[2 * c], z[2 * c + H], cs.x, cs.y, a0, b0);
+            rope_rotate(z[2 * c + 1], z[2 * c + 1 + H], cs.z, cs.w, a1, b1);
+            z[2 * c] = a0;
+            z[2 * c + H] = b0;
+            z[2 * c + 1] = a1;
+            z[2 * c + 1 + H] = b1;
+        }
+    };
+    if (head < p.h_q) {
+        rotate(y);
+        store_row(p.qr + ((static_cast<int64_t>(b) * p.h_q + head) * p.L + pos) * D, y);
+    } else if (head < p.h_q + p.h_kv) {
+        const int u = head - p.h_q;
+        store_row(p.k + ((static_cast<int64_t>(b) * p.L + pos) * p.h_kv + u) * D, y);
+        rotate(y);
+        store_row(p.kr + ((static_cast<int64_t>(b) * p.h_kv + u) * p.L + pos) * D, y);
+    } else {
+        const int u = head - p.h_q - p.h_kv;
+        store_row(p.v + ((static_cast<int64_t>(b) * p.L + pos) * p.h_kv + u) * D, y);
+    }
+}
+
+// ---------------------------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    qkv_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w, const Params p) {
+    extern __shared__ uint8_t dyn_smem_raw[];
+    __shared__ Shared sh;
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dyn_smem_raw) + 1023) & ~uintptr_t(1023));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&sh.full[s], 1);
+            mbar_init(&sh.empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&sh.acc_full[b], 1);
+            mbar_init(&sh.acc_empty[b], 4 * 32);
+        }
+        mbar_init(&sh.mma_done, 1);
+        sh.abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == WARP_MMA) {
+        tmem_alloc(&sh.tmem_base, TMEM_COLS);
+        tmem_relinquish();
+    }
+    if (warp == WARP_TMA && lane == 0) {
+        prefetch_tensormap(&tm_x);
+        prefetch_tensormap(&tm_w);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sh.tmem_base;
+    volatile int* abort = &sh.abort;
+
+    if (warp == WARP_TMA) {
+        // ================================================================ TMA producer
+        if (lane == 0) {
+            uint32_t it = 0;   // K blocks issued (ring position)
+            bool ok = true;
+            for (int tile = blockIdx.x; ok && tile < p.n_tiles; tile += gridDim.x) {
+                const int mt = tile / p.n_ntiles, nt = tile % p.n_ntiles;
+                for (int kb = 0; kb < p.kblocks; ++kb) {
+                    const int s = static_cast<int>(it % STAGES);
+                    if (it >= STAGES && !mbar_wait(&sh.empty[s], ((it / STAGES) - 1) & 1, p.err, abort)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&sh.full[s], STAGE_BYTES);
+                    uint8_t* a = smem + s * STAGE_BYTES;
+                    tma_load_2d(a, &tm_x, &sh.full[s], kb * BK, mt * BM);
+                    tma_load_2d(a + A_BYTES, &tm_w, &sh.full[s], kb * BK, nt * BN);
+                    ++it;
+                }
+            }
+            // Never leave the CTA with copies still landing in its shared memory.
+            for (uint32_t j = (it > STAGES ? it - STAGES : 0); j < it; ++j)
+                mbar_wait(&sh.full[j % STAGES], (j / STAGES) & 1, p.err, nullptr);
+        }
+    } else if (warp == WARP_MMA) {
+        // ================================================================ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN, false);
+            const uint32_t base = smem_u32(smem);
+            uint32_t it = 0;
+            int local = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; ok && tile < p.n_tiles; tile += gridDim.x, ++local) {
+                const int buf = local & 1;
+                // The epilogue must have read this accumulator out (two tiles ago) before it is overwritten.
+                if (local >= 2 && !mbar_wait(&sh.acc_empty[buf], ((local >> 1) - 1) & 1, p.err, abort)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem + static_cast<uint32_t>(buf * BN);
+                for (int kb = 0; kb < p.kblocks; ++kb, ++it) {
+                    const int s = static_cast<int>(it % STAGES);
+                    if (!mbar_wait(&sh.full[s], (it / STAGES) & 1, p.err, abort)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a_addr = base + static_cast<uint32_t>(s * STAGE_BYTES);
+                    const uint32_t b_addr = a_addr + A_BYTES;
+#pragma unroll
+                    for (int kk = 0; kk < BK / 16; ++kk)
+                        umma_ss(d_tmem, sw128_desc(a_addr + kk * 32, 16, 1024), sw128_desc(b_addr + kk * 32, 16, 1024),
+                                IDESC, (kb > 0 || kk > 0) ? 1u : 0u);
+                    umma_commit(&sh.empty[s]);
+                }
+                if (!ok) break;
+                umma_commit(&sh.acc_full[buf]);
+            }
+            // Every MMA must have finished before the tensor memory is released.
+            umma_commit(&sh.mma_done);
+            mbar_wait(&sh.mma_done, 0, p.err, nullptr);
+        }
+    } else {
+        // ================================================================ epilogue (warps 2..5)
+        const int quarter = warp & 3;                       // TMEM lanes 32*quarter .. +31
+        const int r = quarter * 32 + lane;                  // token row within the tile
+        const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
+        int local = 0;
+        for (int tile = blockIdx.x; tile < p.n_tiles; tile += gridDim.x, ++local) {
+            const int buf = local & 1;
+            if (!__all_sync(0xffffffffu, mbar_wait(&sh.acc_full[buf], (local >> 1) & 1, p.err, abort))) break;
+            tc_fence_after();
+            const int mt = tile / p.n_ntiles, nt = tile % p.n_ntiles;
+            const int t = mt * BM + r;
+            const bool valid = t < p.T;
+            const int b = valid ? t / p.L : 0, pos = valid ? t % p.L : 0;
+#pragma unroll 1
+            for (int hh = 0; hh < BN / D; ++hh) {
+                const int n0 = nt * BN + hh * D;
+                if (n0 >= p.N) break;
+                float acc[D];
+#pragma unroll
+                for (int c = 0; c < D / 32; ++c)
+                    tmem_ld32(tmem + lane_base + static_cast<uint32_t>(buf * BN + hh * D + 32 * c),
+                              *reinterpret_cast<uint32_t(*)[32]>(acc + 32 * c));
+                tmem_wait_ld();
+                if (valid) store_head<D>(p, acc, n0, b, pos);
+            }
+            // This thread's reads of the accumulator are complete: release it to the MMA warp.
+            tc_fence_before();
+            mbar_arrive(&sh.acc_empty[buf]);
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == WARP_MMA) {
+        tc_fence_after();
+        tmem_dealloc(tmem, TMEM_COLS);
+    }
+}
+
+}  // namespace qkv
+}  // namespace gqa

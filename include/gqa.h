@@ -142,6 +142,36 @@ GQA_API int gqa_decode_paged(const void* q, const void* kpages, const void* vpag
                              const int* seqlens, void* out, int B, int h_q, int h_kv, int d, int page_size,
                              int num_pages, int max_pages_per_seq, float theta);
 
+/*
+ * gqa_qkv_rope -- the step before the attention, fused (page "Qwen2 architecture introduction",
+ * aicoding.csdn.net, §4.1.3 steps 1-3): the Q, K, V projections with their bias, the split into h_q query
+ * heads and h_kv key/value heads, and RoPE on Q and K; it also writes the KV-cache rows of the sequences.
+ *   x      [B, L, d_model]                 hidden states (after RMSNorm), bf16
+ *   w_qkv  [(h_q + 2 h_kv) d, d_model]     rows 0 .. h_q d - 1 are W_Q^T, then W_K^T, then W_V^T (the
+ *                                          nn.Linear weight layout: output feature major), bf16
+ *   b_qkv  [(h_q + 2 h_kv) d]              the matching bias, bf16, or NULL for none
+ * Outputs (bf16, caller-owned): with Y = x w_qkv^T + b_qkv split into heads, at positions 0 .. L-1,
+ *   qr [B, h_q, L, d]   rotated Q, head-major      kr [B, h_kv, L, d]   rotated K, head-major
+ *   k  [B, L, h_kv, d]  un-rotated K, token-major  v  [B, L, h_kv, d]   V, token-major
+ * k and v are exactly the packed cache rows of gqa_decode for B sequences of L rows stored back to back,
+ * so pointing them into a cache appends the sequences; qr, kr and v are the inputs of
+ * gqa_prefill_rotated.  Each output element is the fp32 accumulation rounded to bf16 once.
+ * d in {64, 128}; d_model a positive multiple of 8; all pointers 16-byte aligned.  B == 0 or L == 0 is a
+ * no-op.  Uses an internal device table of cos / sin for positions 0 .. L-1 (L * d/2 * 8 bytes), rebuilt
+ * when L, d or theta change and kept until gqa_release().
+ */
+GQA_API int gqa_qkv_rope(const void* x, const void* w_qkv, const void* b_qkv, void* qr, void* kr, void* k, void* v,
+                         int B, int L, int d_model, int h_q, int h_kv, int d, float theta);
+
+/*
+ * gqa_prefill_rotated -- the causal attention of gqa_prefill on inputs that are already rotated (page
+ * "Qwen2 architecture introduction", §4.1.3 steps 4-5): qr [B, h_q, L, d] and kr [B, h_kv, L, d]
+ * head-major as gqa_qkv_rope writes them, v [B, L, h_kv, d], out [B, L, h_q, d].  No RoPE and no
+ * workspace: the prep pass of gqa_prefill is skipped.  Same checks and conventions as gqa_prefill.
+ */
+GQA_API int gqa_prefill_rotated(const void* qr, const void* kr, const void* v, void* out, int B, int L, int h_q,
+                                int h_kv, int d);
+
 /* Stream for subsequent calls (a cudaStream_t passed as void*; NULL = legacy stream). */
 GQA_API int gqa_set_stream(void* cuda_stream);
 
@@ -152,7 +182,7 @@ GQA_API int gqa_set_stream(void* cuda_stream);
  */
 GQA_API int gqa_last_error(void);
 
-/* Frees the internal workspaces of every device this process used (synchronises each). */
+/* Frees the internal workspaces (and the cos / sin table) of every device this process used (synchronises each). */
 GQA_API void gqa_release(void);
 
 /* Static, human-readable text for a GQA_ERR_* code. */

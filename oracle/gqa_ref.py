@@ -214,12 +214,13 @@ def decode_paged_ref(q, kpages, vpages, block_table, seqlens, theta: float, batc
     return np.stack(outs, axis=0)
 
 
-def qkv_rope_ref(x, w_qkv, b_qkv, h_q: int, h_kv: int, d: int, theta: float):
+def qkv_rope_ref(x, w_qkv, b_qkv, h_q: int, h_kv: int, d: int, theta: float, positions=None):
     """Steps 1-3 of the aicoding.csdn.net page, §4.1.3: projections with bias, split into heads, RoPE.
 
     x [B, L, d_model]; w_qkv [(h_q + 2 h_kv) d, d_model] holds the rows of W_Q^T, W_K^T, W_V^T (so the
     projection is x @ w_qkv^T, i.e. X W with W = w_qkv^T); b_qkv [(h_q + 2 h_kv) d] or None.  Positions
-    are 0 .. L-1 in every batch row.  Returns float64 arrays in the layouts the CUDA path writes:
+    are 0 .. L-1 in every batch row (or the given `positions` [L], for checking sampled rows of a longer
+    sequence).  Returns float64 arrays in the layouts the CUDA path writes:
     qr [B, h_q, L, d] and kr [B, h_kv, L, d] rotated (head-major), k and v [B, L, h_kv, d] un-rotated
     (token-major: the packed cache rows of the sequence).
     """
@@ -231,7 +232,7 @@ def qkv_rope_ref(x, w_qkv, b_qkv, h_q: int, h_kv: int, d: int, theta: float):
     q = y[..., :h_q * d].reshape(B, L, h_q, d)
     k = y[..., h_q * d:(h_q + h_kv) * d].reshape(B, L, h_kv, d)
     v = y[..., (h_q + h_kv) * d:].reshape(B, L, h_kv, d)
-    pos = np.arange(L)
+    pos = np.arange(L) if positions is None else np.asarray(positions)
     qr = np.stack([rope(q[b], pos, theta) for b in range(B)]).transpose(0, 2, 1, 3)
     kr = np.stack([rope(k[b], pos, theta) for b in range(B)]).transpose(0, 2, 1, 3)
     return qr, kr, k, v

@@ -123,3 +123,14 @@ def test_qkv_inputs_shapes_scales_and_determinism():
     assert bool((x == x2).all()) and bool((wq == wq2).all()) and bool((b == b2).all())
     assert 0.8 < float(wq.float().std()) * 16 < 1.2   # std 1/sqrt(d_model)
     assert gi.qkv_inputs(w, d_model=256, bias=False)[2] is None
+
+
+def test_explicit_positions_match_the_full_sequence():
+    x, w, b, h_q, h_kv, d = _case(B=1, L=9, seed=8)
+    full = R.qkv_rope_ref(x, w, b, h_q, h_kv, d, THETA)
+    rows = [0, 4, 8]
+    part = R.qkv_rope_ref(x[:, rows], w, b, h_q, h_kv, d, THETA, positions=rows)
+    np.testing.assert_allclose(part[0], full[0][:, :, rows], atol=1e-12)
+    np.testing.assert_allclose(part[1], full[1][:, :, rows], atol=1e-12)
+    np.testing.assert_allclose(part[2], full[2][:, rows], atol=1e-12)
+    np.testing.assert_allclose(part[3], full[3][:, rows], atol=1e-12)
