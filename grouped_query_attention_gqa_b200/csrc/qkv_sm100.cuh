@@ -11,7 +11,8 @@
 // 256 output columns = 2 heads of d = 128 or 4 of d = 64):
 //   warp 0     TMA producer: 64-wide K blocks of X (128 x 64) and W (256 x 64) into a 4-stage ring
 //   warp 1     MMA issuer: 4 x tcgen05.mma M128 N256 K16 per K block into one of two TMEM accumulators
-//   warps 2-5  epilogue: one TMEM lane (token row) per thread; per head: + bias, rotate, round, store
+//   warps 2-5  epilogue: one TMEM lane (token row) per thread; per head: + bias, rotate, round, and
+//              store through a per-warp shared-memory staging buffer as whole rows
 // The two accumulators (2 x 256 TMEM columns) let the epilogue of one tile overlap the main loop of the
 // next.  cos / sin come from a per-position table built once per (L, d, theta).
 #pragma once
@@ -37,7 +38,9 @@ constexpr int WARP_TMA = 0, WARP_MMA = 1;
 constexpr int A_BYTES = BM * BK * 2;     // 16 KB
 constexpr int B_BYTES = BN * BK * 2;     // 32 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr int DYN = STAGES * STAGE_BYTES + 1024;
+constexpr int EPI_WARPS = 4;
+constexpr int STAGING = 32 * 128 * 2;    // one epilogue warp's 32 rows of up to 128 bf16
+constexpr int DYN = STAGES * STAGE_BYTES + EPI_WARPS * STAGING + 1024;
 constexpr int TMEM_COLS = 2 * BN;
 constexpr int TABLE_THREADS = 256;
 
@@ -78,8 +81,39 @@ __global__ void __launch_bounds__(TABLE_THREADS) rope_table_kernel(float2* __res
 
 // ---------------------------------------------------------------------------------------------
 // One head (D columns starting at n0) of one token row, in place: + bias, rotate if Q or K, round, store.
+// One output row per lane (dst, nullptr for a row past the end), D values in z: round to bf16 and store the
+// warp's 32 rows through its shared-memory staging buffer, so that each global store instruction writes
+// whole rows (D * 2 bytes each) instead of one 16-byte piece of 32 different rows.  Chunk c of row r is
+// staged at chunk position c ^ (r mod CH): writing (one row per lane) and reading (CH lanes per row) are
+// both free of bank conflicts.
 template <int D>
-__device__ __forceinline__ void store_head(const Params& p, float (&y)[D], int n0, int b, int pos) {
+__device__ __forceinline__ void store_rows(uint8_t* stage, __nv_bfloat16* dst, const float* z, int lane) {
+    constexpr int CH = D / 8;             // 16-byte chunks per row
+    constexpr int RPI = 32 / CH;          // rows per store instruction
+    uint4* st = reinterpret_cast<uint4*>(stage);
+#pragma unroll
+    for (int c = 0; c < CH; ++c)
+        st[lane * CH + (c ^ (lane & (CH - 1)))] =
+            make_uint4(pack_bf16x2(z[8 * c], z[8 * c + 1]), pack_bf16x2(z[8 * c + 2], z[8 * c + 3]),
+                       pack_bf16x2(z[8 * c + 4], z[8 * c + 5]), pack_bf16x2(z[8 * c + 6], z[8 * c + 7]));
+    __syncwarp();
+    const uint64_t mine = reinterpret_cast<uint64_t>(dst);
+    const int c = lane % CH;
+#pragma unroll
+    for (int j = 0; j < 32 / RPI; ++j) {
+        const int r = j * RPI + lane / CH;
+        const uint64_t row = __shfl_sync(0xffffffffu, mine, r);
+        const uint4 val = st[r * CH + (c ^ (r & (CH - 1)))];
+        if (row) reinterpret_cast<uint4*>(row)[c] = val;
+    }
+    __syncwarp();   // the buffer is reused by the next call
+}
+
+// One head (D columns starting at n0) of one token row per lane, in place: + bias, rotate if Q or K, then
+// the row goes to its output(s).  Lanes with valid == false (rows past the end) take part without storing.
+template <int D>
+__device__ __forceinline__ void store_head(const Params& p, float (&y)[D], int n0, int b, int pos, bool valid,
+                                           uint8_t* stage, int lane) {
     constexpr int H = D / 2;
     if (p.bias) {
         const uint4* bb = reinterpret_cast<const uint4*>(p.bias + n0);
@@ -95,38 +129,48 @@ __device__ __forceinline__ void store_head(const Params& p, float (&y)[D], int n
         }
     }
     const int head = n0 / D;
-    auto store_row = [&](__nv_bfloat16* dst, const float* z) {
-        uint4* o = reinterpret_cast<uint4*>(dst);
-#pragma unroll
-        for (int c = 0; c < D / 8; ++c)
-            o[c] = make_uint4(pack_bf16x2(z[8 * c], z[8 * c + 1]), pack_bf16x2(z[8 * c + 2], z[8 * c + 3]),
-                              pack_bf16x2(z[8 * c + 4], z[8 * c + 5]), pack_bf16x2(z[8 * c + 6], z[8 * c + 7]));
-    };
+    // Rotation pairs (i, i + H): the (cos, sin) of a row's H frequencies are read from the table in
+    // chunks of 16 frequencies (8 float4), the next chunk's loads issued before the current chunk is
+    // rotated, so at most two chunks are live in registers beside the row.
+    constexpr int CHUNK = 16;
+    constexpr int NCH = H / CHUNK;
+    const float4* trow = reinterpret_cast<const float4*>(p.tab + static_cast<int64_t>(pos) * H);
     auto rotate = [&](float* z) {
-        const float4* t = reinterpret_cast<const float4*>(p.tab + static_cast<int64_t>(pos) * H);
+        float4 tb[2][CHUNK / 2];
 #pragma unroll
-        for (int c = 0; c < H / 2; ++c) {
-            const float4 cs = t[c];   // (cos, sin) of frequencies 2c and 2c + 1
-            float a0, b0, a1, b1;
-            rope_rotate(z[2 * c], z[2 * c + H], cs.x, cs.y, a0, b0);
-            rope_rotate(z[2 * c + 1], z[2 * c + 1 + H], cs.z, cs.w, a1, b1);
-            z[2 * c] = a0;
-            z[2 * c + H] = b0;
-            z[2 * c + 1] = a1;
-            z[2 * c + 1 + H] = b1;
+        for (int c = 0; c < CHUNK / 2; ++c) tb[0][c] = trow[c];
+#pragma unroll
+        for (int ch = 0; ch < NCH; ++ch) {
+            if (ch + 1 < NCH) {
+#pragma unroll
+                for (int c = 0; c < CHUNK / 2; ++c) tb[(ch + 1) & 1][c] = trow[(ch + 1) * (CHUNK / 2) + c];
+            }
+#pragma unroll
+            for (int c = 0; c < CHUNK / 2; ++c) {
+                const float4 cs = tb[ch & 1][c];   // (cos, sin) of frequencies i and i + 1
+                const int i = ch * CHUNK + 2 * c;
+                float a0, b0, a1, b1;
+                rope_rotate(z[i], z[i + H], cs.x, cs.y, a0, b0);
+                rope_rotate(z[i + 1], z[i + 1 + H], cs.z, cs.w, a1, b1);
+                z[i] = a0;
+                z[i + H] = b0;
+                z[i + 1] = a1;
+                z[i + 1 + H] = b1;
+            }
         }
     };
+    auto row_of = [&](__nv_bfloat16* base, int64_t idx) { return valid ? base + idx * D : nullptr; };
     if (head < p.h_q) {
         rotate(y);
-        store_row(p.qr + ((static_cast<int64_t>(b) * p.h_q + head) * p.L + pos) * D, y);
+        store_rows<D>(stage, row_of(p.qr, (static_cast<int64_t>(b) * p.h_q + head) * p.L + pos), y, lane);
     } else if (head < p.h_q + p.h_kv) {
         const int u = head - p.h_q;
-        store_row(p.k + ((static_cast<int64_t>(b) * p.L + pos) * p.h_kv + u) * D, y);
+        store_rows<D>(stage, row_of(p.k, (static_cast<int64_t>(b) * p.L + pos) * p.h_kv + u), y, lane);
         rotate(y);
-        store_row(p.kr + ((static_cast<int64_t>(b) * p.h_kv + u) * p.L + pos) * D, y);
+        store_rows<D>(stage, row_of(p.kr, (static_cast<int64_t>(b) * p.h_kv + u) * p.L + pos), y, lane);
     } else {
         const int u = head - p.h_q - p.h_kv;
-        store_row(p.v + ((static_cast<int64_t>(b) * p.L + pos) * p.h_kv + u) * D, y);
+        store_rows<D>(stage, row_of(p.v, (static_cast<int64_t>(b) * p.L + pos) * p.h_kv + u), y, lane);
     }
 }
 
@@ -234,6 +278,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int quarter = warp & 3;                       // TMEM lanes 32*quarter .. +31
         const int r = quarter * 32 + lane;                  // token row within the tile
         const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
+        uint8_t* stage = smem + STAGES * STAGE_BYTES + (warp - 2) * STAGING;
         int local = 0;
         for (int tile = blockIdx.x; tile < p.n_tiles; tile += gridDim.x, ++local) {
             const int buf = local & 1;
@@ -253,7 +298,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     tmem_ld32(tmem + lane_base + static_cast<uint32_t>(buf * BN + hh * D + 32 * c),
                               *reinterpret_cast<uint32_t(*)[32]>(acc + 32 * c));
                 tmem_wait_ld();
-                if (valid) store_head<D>(p, acc, n0, b, pos);
+                store_head<D>(p, acc, n0, b, pos, valid, stage, lane);
             }
             // This thread's reads of the accumulator are complete: release it to the MMA warp.
             tc_fence_before();
