@@ -120,6 +120,24 @@ def qkv_inputs(w: Workload, d_model: int | None = None, device: str = "cpu", bia
     return x, wq, b
 
 
+def out_proj_inputs(w: Workload, d_model: int | None = None, device: str = "cpu"):
+    """Synthetic inputs of the output projection for the prefill workload w: attn [B*L, h_q*d] ~ N(0, 1)
+    (the concatenated heads), w_o [d_model, h_q*d] ~ N(0, 1/(h_q*d)) (nn.Linear layout), residual
+    [B*L, d_model] ~ N(0, 1).  All bf16."""
+    assert w.kind == "prefill"
+    dm = d_model or D_MODEL[(w.h_q, w.h_kv, w.d)]
+    k = w.h_q * w.d
+    gen = _gen(w.seed + 4242, device)
+    attn = _randn_bf16((w.B * w.L, k), gen, device)
+    wo = torch.empty((dm, k), dtype=torch.bfloat16, device=device)
+    for s0 in range(0, dm, 1024):
+        e = min(dm, s0 + 1024)
+        wo[s0:e] = (torch.randn((e - s0, k), generator=gen, dtype=torch.float32, device=device)
+                    / (k ** 0.5)).to(torch.bfloat16)
+    res = _randn_bf16((w.B * w.L, dm), gen, device)
+    return attn, wo, res
+
+
 def decode_inputs(w: Workload, device: str = "cpu", seqlens=None):
     """seqlens int32 [B]; q [B,h_q,d]; kcache, vcache packed [sum(seqlens), h_kv, d].
 

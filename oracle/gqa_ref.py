@@ -39,6 +39,9 @@ into independent blocks (each block is still the full materialised product):
      the hidden states times W_Q, W_K, W_V plus the bias, split into h_q and
      h_kv heads; Q and K are then rotated as in step 1.
      ``qkv_rope_ref`` writes it out with one matrix product.
+  7. Output projection and residual (aicoding.csdn.net page, §4.1.3 steps
+     5-6): the concatenated heads times W_O, plus the sub-layer input.
+     ``out_proj_ref``.
 
 Every function is pinned by ``tests/test_oracle_pins.py`` against closed forms,
 invariants the pages state and a brute-force restatement.
@@ -236,6 +239,19 @@ def qkv_rope_ref(x, w_qkv, b_qkv, h_q: int, h_kv: int, d: int, theta: float, pos
     qr = np.stack([rope(q[b], pos, theta) for b in range(B)]).transpose(0, 2, 1, 3)
     kr = np.stack([rope(k[b], pos, theta) for b in range(B)]).transpose(0, 2, 1, 3)
     return qr, kr, k, v
+
+
+def out_proj_ref(attn, w_o, residual=None) -> np.ndarray:
+    """Steps 5-6 of the aicoding.csdn.net page, §4.1.3: Concat of the heads times W_O, plus the residual.
+
+    attn [T, h_q * d] is the concatenated heads (the prefill output [B, L, h_q, d] viewed as rows);
+    w_o [d_model, h_q * d] holds the rows of W_O^T (nn.Linear layout), so AttnOut = attn @ w_o^T;
+    residual [T, d_model] (the sub-layer input X_in) or None.  Returns float64 [T, d_model].
+    """
+    y = as_f64(attn) @ as_f64(w_o).T
+    if residual is not None:
+        y = y + as_f64(residual)
+    return y
 
 
 def qkv_flops(B: int, L: int, d_model: int, h_q: int, h_kv: int, d: int) -> float:

@@ -134,3 +134,50 @@ def test_explicit_positions_match_the_full_sequence():
     np.testing.assert_allclose(part[1], full[1][:, :, rows], atol=1e-12)
     np.testing.assert_allclose(part[2], full[2][:, rows], atol=1e-12)
     np.testing.assert_allclose(part[3], full[3][:, rows], atol=1e-12)
+
+
+# ---------------------------------------------------------------- output projection + residual
+def _brute_out(attn, w_o, res):
+    T, k = attn.shape
+    n = w_o.shape[0]
+    return np.array([[sum(attn[t, kk] * w_o[c, kk] for kk in range(k)) + (res[t, c] if res is not None else 0.0)
+                      for c in range(n)] for t in range(T)])
+
+
+def _out_pins_pass(fn):
+    try:
+        rng = np.random.default_rng(21)
+        for T, k, n in [(5, 8, 6), (3, 12, 4)]:
+            attn, w_o, res = rng.standard_normal((T, k)), rng.standard_normal((n, k)), rng.standard_normal((T, n))
+            for r_ in (res, None):
+                if not np.allclose(fn(attn, w_o, r_), _brute_out(attn, w_o, r_), atol=1e-12):
+                    return False
+        return True
+    except Exception:
+        return False
+
+
+def test_out_proj_ref_matches_brute_force():
+    assert _out_pins_pass(R.out_proj_ref)
+
+
+def test_out_proj_of_the_attention_output_is_concat_times_w_o():
+    """The prefill output [B, L, h_q, d] viewed as rows is the Concat of step 5: head t occupies columns
+    t*d .. t*d + d - 1, so projecting it equals summing per-head products with the column blocks of W_O."""
+    rng = np.random.default_rng(5)
+    B, L, h_q, h_kv, d, dm = 1, 6, 4, 2, 8, 10
+    q, k, v = (rng.standard_normal((B, L, h, d)) for h in (h_q, h_kv, h_kv))
+    heads = R.prefill_ref(q, k, v, THETA)
+    w_o = rng.standard_normal((dm, h_q * d))
+    got = R.out_proj_ref(heads.reshape(B * L, h_q * d), w_o)
+    per_head = sum(heads[0, :, t] @ w_o[:, t * d:(t + 1) * d].T for t in range(h_q))
+    np.testing.assert_allclose(got, per_head, atol=1e-12)
+
+
+@pytest.mark.parametrize("fn", [
+    lambda a, w, r: R.out_proj_ref(a, w, None),                  # residual dropped
+    lambda a, w, r: a @ w[:, ::-1].T + (0 if r is None else r),    # columns of W_O reversed
+    lambda a, w, r: R.out_proj_ref(a, w, r) - (0 if r is None else 2 * r),   # residual subtracted
+])
+def test_out_proj_pins_catch_planted_mistakes(fn):
+    assert not _out_pins_pass(fn)
