@@ -49,6 +49,8 @@ def load() -> ctypes.CDLL:
     lib.gqa_qkv_rope.restype = i
     lib.gqa_prefill_rotated.argtypes = [vp, vp, vp, vp, i, i, i, i, i]
     lib.gqa_prefill_rotated.restype = i
+    lib.gqa_out_proj.argtypes = [vp, vp, vp, vp, i, i, i]
+    lib.gqa_out_proj.restype = i
     lib.gqa_set_timing_events.argtypes = [vp, vp]
     lib.gqa_set_timing_events.restype = i
     lib.gqa_set_stream.argtypes = [vp]
@@ -216,6 +218,30 @@ def prefill_rotated(qr: torch.Tensor, kr: torch.Tensor, v: torch.Tensor, out: to
         rc = load().gqa_prefill_rotated(_ptr(qr), _ptr(kr), _ptr(v), _ptr(out), B, L, h_q, h_kv, d)
     if rc != GQA_OK:
         raise GQAError(rc, "gqa_prefill_rotated")
+    return out
+
+
+def out_proj(attn: torch.Tensor, w_o: torch.Tensor, residual: torch.Tensor | None = None,
+             out: torch.Tensor | None = None) -> torch.Tensor:
+    """out [T, d_model] = attn [T, d_in] @ w_o[d_model, d_in]^T (+ residual [T, d_model]); `out` may be
+    `residual` itself.  A [B, L, h_q, d] attention output may be passed as attn (viewed as [B*L, h_q*d])."""
+    a = attn.reshape(-1, attn.shape[-2] * attn.shape[-1]) if attn.dim() == 4 else attn
+    if a.dim() != 2 or w_o.dim() != 2:
+        raise ValueError("attn must be [T, d_in] (or [B, L, h, d]) and w_o [d_model, d_in]")
+    T, d_in = a.shape
+    dm = w_o.shape[0]
+    _check(a, "attn", None)
+    _check(w_o, "w_o", (dm, d_in))
+    if residual is not None:
+        _check(residual, "residual", (T, dm))
+    if out is None:
+        out = a.new_empty(T, dm)
+    _check(out, "out", (T, dm))
+    with torch.cuda.device(a.device):
+        _stream(a.device)
+        rc = load().gqa_out_proj(_ptr(a), _ptr(w_o), _ptr(residual), _ptr(out), T, d_in, dm)
+    if rc != GQA_OK:
+        raise GQAError(rc, "gqa_out_proj")
     return out
 
 

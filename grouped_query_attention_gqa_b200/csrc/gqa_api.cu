@@ -51,6 +51,10 @@ struct DeviceState {
     const void* qkv_key[2] = {nullptr, nullptr};
     long long qkv_dims[3] = {0, 0, 0};
     CUtensorMap qkv_maps[2];
+    bool proj_ready = false;
+    const void* proj_key[2] = {nullptr, nullptr};
+    long long proj_dims[3] = {0, 0, 0};
+    CUtensorMap proj_maps[2];
 };
 
 DeviceState g_dev[kMaxDevices];
@@ -312,6 +316,8 @@ int launch_qkv(DeviceState* st, const void* x, const void* w, const void* bias, 
         st->qkv_dims[2] = d_model;
     }
     Params p;
+    p.resid = nullptr;
+    p.out = nullptr;
     p.bias = static_cast<const __nv_bfloat16*>(bias);
     p.tab = static_cast<const float2*>(st->tab);
     p.qr = static_cast<__nv_bfloat16*>(qr);
@@ -338,6 +344,52 @@ int launch_qkv(DeviceState* st, const void* x, const void* w, const void* bias, 
     const int grid = p.n_tiles < st->num_sms ? p.n_tiles : st->num_sms;
     mark(g_ev_start);
     qkv_kernel<D><<<grid, NUM_THREADS, DYN, g_stream>>>(st->qkv_maps[0], st->qkv_maps[1], p);
+    if (cudaGetLastError() != cudaSuccess) return GQA_ERR_LAUNCH;
+    mark(g_ev_stop);
+    return GQA_OK;
+}
+
+// Output projection + residual: out [T, d_model] = attn [T, d_in] w_o [d_model, d_in]^T (+ resid).
+int launch_proj(DeviceState* st, const void* attn, const void* w_o, const void* resid, void* out, int T, int d_in,
+                int d_model) {
+    using namespace gqa::qkv;
+    if (!get_encoder()) return GQA_ERR_LAUNCH;
+    if (st->proj_key[0] != attn || st->proj_key[1] != w_o || st->proj_dims[0] != T || st->proj_dims[1] != d_in ||
+        st->proj_dims[2] != d_model) {
+        st->proj_key[0] = st->proj_key[1] = nullptr;
+        const cuuint64_t sx[1] = {static_cast<cuuint64_t>(d_in) * 2};
+        const cuuint64_t da[2] = {static_cast<cuuint64_t>(d_in), static_cast<cuuint64_t>(T)};
+        const cuuint32_t ba[2] = {BK, BM};
+        if (!encode_bf16(&st->proj_maps[0], const_cast<void*>(attn), 2, da, sx, ba)) return GQA_ERR_LAUNCH;
+        const cuuint64_t dw[2] = {static_cast<cuuint64_t>(d_in), static_cast<cuuint64_t>(d_model)};
+        const cuuint32_t bw[2] = {BK, BN};
+        if (!encode_bf16(&st->proj_maps[1], const_cast<void*>(w_o), 2, dw, sx, bw)) return GQA_ERR_LAUNCH;
+        st->proj_key[0] = attn;
+        st->proj_key[1] = w_o;
+        st->proj_dims[0] = T;
+        st->proj_dims[1] = d_in;
+        st->proj_dims[2] = d_model;
+    }
+    Params p = {};
+    p.resid = static_cast<const __nv_bfloat16*>(resid);
+    p.out = static_cast<__nv_bfloat16*>(out);
+    p.T = T;
+    p.L = T;
+    p.N = d_model;
+    p.n_ntiles = (d_model + BN - 1) / BN;
+    const long long mtiles = (static_cast<long long>(T) + BM - 1) / BM;
+    if (mtiles * p.n_ntiles > 0x7fffffffLL) return GQA_ERR_DIMS;
+    p.n_tiles = static_cast<int>(mtiles * p.n_ntiles);
+    p.kblocks = (d_in + BK - 1) / BK;
+    p.err = st->err;
+    if (!st->proj_ready) {
+        if (cudaFuncSetAttribute(proj_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, DYN) != cudaSuccess)
+            return GQA_ERR_LAUNCH;
+        st->proj_ready = true;
+    }
+    const int grid = p.n_tiles < st->num_sms ? p.n_tiles : st->num_sms;
+    mark(g_ev_start);
+    proj_kernel<<<grid, NUM_THREADS, DYN, g_stream>>>(st->proj_maps[0], st->proj_maps[1], p);
     if (cudaGetLastError() != cudaSuccess) return GQA_ERR_LAUNCH;
     mark(g_ev_stop);
     return GQA_OK;
@@ -587,6 +639,18 @@ int gqa_qkv_rope(const void* x, const void* w_qkv, const void* b_qkv, void* qr, 
     if (!st) return rc;
     return d == 64 ? launch_qkv<64>(st, x, w_qkv, b_qkv, qr, kr, k, v, B, L, d_model, h_q, h_kv, theta)
                    : launch_qkv<128>(st, x, w_qkv, b_qkv, qr, kr, k, v, B, L, d_model, h_q, h_kv, theta);
+}
+
+int gqa_out_proj(const void* attn, const void* w_o, const void* residual, void* out, int T, int d_in, int d_model) {
+    if (T < 0 || d_in <= 0 || d_in % 8 != 0 || d_model <= 0 || d_model % 128 != 0) return GQA_ERR_DIMS;
+    if (T == 0) return GQA_OK;
+    if (!attn || !w_o || !out) return GQA_ERR_NULL;
+    if (!aligned16(attn) || !aligned16(w_o) || !aligned16(out) || (residual && !aligned16(residual)))
+        return GQA_ERR_ALIGN;
+    int rc = GQA_OK;
+    DeviceState* st = device_state(&rc);
+    if (!st) return rc;
+    return launch_proj(st, attn, w_o, residual, out, T, d_in, d_model);
 }
 
 int gqa_prefill_rotated(const void* qr, const void* kr, const void* v, void* out, int B, int L, int h_q, int h_kv,

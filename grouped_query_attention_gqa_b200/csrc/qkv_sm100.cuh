@@ -8,7 +8,8 @@
 //   v  [B, L, h_kv, d]  V, token-major (cache rows; the attention kernel reads V in this layout)
 //
 // qkv_kernel is a persistent tcgen05 GEMM, one CTA per SM, over 128 x 256 output tiles (128 tokens,
-// 256 output columns = 2 heads of d = 128 or 4 of d = 64):
+// 256 output columns = 2 heads of d = 128 or 4 of d = 64); proj_kernel is the same GEMM with the output
+// projection's epilogue (+ residual, page §4.1.3 steps 5-6):
 //   warp 0     TMA producer: 64-wide K blocks of X (128 x 64) and W (256 x 64) into a 4-stage ring
 //   warp 1     MMA issuer: 4 x tcgen05.mma M128 N256 K16 per K block into one of two TMEM accumulators
 //   warps 2-5  epilogue: one TMEM lane (token row) per thread; per head: + bias, rotate, round, and
@@ -51,6 +52,8 @@ struct Params {
     __nv_bfloat16* kr;
     __nv_bfloat16* k;
     __nv_bfloat16* v;
+    const __nv_bfloat16* resid;  // output projection: residual [T, N] or nullptr
+    __nv_bfloat16* out;          // output projection: out [T, N] (may be resid itself)
     int T, L, N, h_q, h_kv;
     int n_ntiles, n_tiles, kblocks;
     int* err;
@@ -174,10 +177,32 @@ __device__ __forceinline__ void store_head(const Params& p, float (&y)[D], int n
     }
 }
 
+// The output projection's epilogue: 128 columns of one row per lane, + the residual, stored as rows.
+__device__ __forceinline__ void store_resid(const Params& p, float (&y)[128], int n0, int t, bool valid,
+                                            uint8_t* stage, int lane) {
+    if (p.resid && valid) {
+        const uint4* rr = reinterpret_cast<const uint4*>(p.resid + static_cast<int64_t>(t) * p.N + n0);
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+            const uint4 w = rr[c];
+            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                y[8 * c + 2 * e] += bf16lo_to_f32(ws[e]);
+                y[8 * c + 2 * e + 1] += bf16hi_to_f32(ws[e]);
+            }
+        }
+    }
+    store_rows<128>(stage, valid ? p.out + static_cast<int64_t>(t) * p.N + n0 : nullptr, y, lane);
+}
+
+enum Epilogue { kQKV = 0, kResidual = 1 };
+
 // ---------------------------------------------------------------------------------------------
-template <int D>
-__global__ void __launch_bounds__(NUM_THREADS, 1)
-    qkv_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w, const Params p) {
+// The persistent GEMM: Y[T, N] = X[T, K] W[N, K]^T with the epilogue EPI.  For kQKV, D is the head size
+// (tiles are processed head by head); for kResidual, D = 128 (tiles are processed 128 columns at a time).
+template <int D, int EPI>
+__device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtensorMap& tm_w, const Params& p) {
     extern __shared__ uint8_t dyn_smem_raw[];
     __shared__ Shared sh;
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dyn_smem_raw) + 1023) & ~uintptr_t(1023));
@@ -298,7 +323,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     tmem_ld32(tmem + lane_base + static_cast<uint32_t>(buf * BN + hh * D + 32 * c),
                               *reinterpret_cast<uint32_t(*)[32]>(acc + 32 * c));
                 tmem_wait_ld();
-                store_head<D>(p, acc, n0, b, pos, valid, stage, lane);
+                if (EPI == kQKV) store_head<D>(p, acc, n0, b, pos, valid, stage, lane);
+                else store_resid(p, *reinterpret_cast<float(*)[128]>(acc), n0, t, valid, stage, lane);
             }
             // This thread's reads of the accumulator are complete: release it to the MMA warp.
             tc_fence_before();
@@ -312,6 +338,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tc_fence_after();
         tmem_dealloc(tmem, TMEM_COLS);
     }
+}
+
+template <int D>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    qkv_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w, const Params p) {
+    gemm_body<D, kQKV>(tm_x, tm_w, p);
+}
+
+// Output projection + residual (page "Qwen2 architecture introduction", §4.1.3 steps 5-6):
+// out = attn W_O + X_in, with attn the concatenated heads [T, h_q d] and W_O^T [d_model, h_q d].
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    proj_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w, const Params p) {
+    gemm_body<128, kResidual>(tm_x, tm_w, p);
 }
 
 }  // namespace qkv

@@ -172,6 +172,20 @@ GQA_API int gqa_qkv_rope(const void* x, const void* w_qkv, const void* b_qkv, vo
 GQA_API int gqa_prefill_rotated(const void* qr, const void* kr, const void* v, void* out, int B, int L, int h_q,
                                 int h_kv, int d);
 
+/*
+ * gqa_out_proj -- the step after the attention (page "Qwen2 architecture introduction", §4.1.3 steps 5-6):
+ * the concatenated heads times W_O, plus the residual:  out = attn w_o^T + residual.
+ *   attn     [T, d_in]       the attention output viewed as rows: gqa_prefill's out [B, L, h_q, d] is
+ *                            already this Concat with T = B*L, d_in = h_q d
+ *   w_o      [d_model, d_in] rows of W_O^T (the nn.Linear weight layout), bf16
+ *   residual [T, d_model]    the sub-layer input X_in, or NULL for none
+ *   out      [T, d_model]    may be the same buffer as residual (updated in place)
+ * Each element is the fp32 accumulation (plus the residual in fp32) rounded once to bf16.  d_in a positive
+ * multiple of 8, d_model a positive multiple of 128, pointers 16-byte aligned; T == 0 is a no-op.
+ */
+GQA_API int gqa_out_proj(const void* attn, const void* w_o, const void* residual, void* out, int T, int d_in,
+                         int d_model);
+
 /* Stream for subsequent calls (a cudaStream_t passed as void*; NULL = legacy stream). */
 GQA_API int gqa_set_stream(void* cuda_stream);
 

@@ -31,7 +31,8 @@ def codes():
 
 def test_header_declares_the_entry_points():
     names = set(declared())
-    for n in ["gqa_prefill", "gqa_decode", "gqa_decode_paged", "gqa_set_stream", "gqa_last_error", "gqa_release",
+    for n in ["gqa_prefill", "gqa_decode", "gqa_decode_paged", "gqa_qkv_rope", "gqa_prefill_rotated",
+              "gqa_out_proj", "gqa_set_stream", "gqa_last_error", "gqa_release",
               "gqa_strerror", "gqa_abi_version", "gqa_set_timing_events"]:
         assert n in names
 
@@ -111,6 +112,50 @@ def paged_args(q=P16, kp=P16, vp=P16, bt=P16, s=P16, out=P16, B=4, h_q=28, h_kv=
 ])
 def test_decode_paged_validation(lib, args, code):
     assert lib.gqa_decode_paged(*args) == codes()[code]
+
+
+def qkv_args(x=P16, w=P16, b=None, qr=P16, kr=P16, k=P16, v=P16, B=1, L=16, dm=256, h_q=28, h_kv=4, d=128, theta=F):
+    return (x, w, b, qr, kr, k, v, B, L, dm, h_q, h_kv, d, theta)
+
+
+@pytest.mark.parametrize("args,code", [
+    (qkv_args(B=-1), "GQA_ERR_DIMS"),
+    (qkv_args(dm=0), "GQA_ERR_DIMS"),
+    (qkv_args(dm=100), "GQA_ERR_DIMS"),          # not a multiple of 8
+    (qkv_args(h_kv=3), "GQA_ERR_DIMS"),
+    (qkv_args(d=96), "GQA_ERR_HEAD_DIM"),
+    (qkv_args(theta=ctypes.c_float(-2.0)), "GQA_ERR_THETA"),
+    (qkv_args(x=None), "GQA_ERR_NULL"),
+    (qkv_args(v=None), "GQA_ERR_NULL"),
+    (qkv_args(b=ctypes.c_void_p(264)), "GQA_ERR_ALIGN"),
+    (qkv_args(kr=ctypes.c_void_p(8)), "GQA_ERR_ALIGN"),
+    (qkv_args(x=None, w=None, qr=None, kr=None, k=None, v=None, L=0), "GQA_OK"),
+])
+def test_qkv_rope_validation(lib, args, code):
+    assert lib.gqa_qkv_rope(*args) == codes()[code]
+
+
+@pytest.mark.parametrize("args,code", [
+    ((P16, P16, P16, P16, -1, 16, 28, 4, 128), "GQA_ERR_DIMS"),
+    ((P16, P16, P16, P16, 1, 16, 28, 4, 80), "GQA_ERR_HEAD_DIM"),
+    ((P16, None, P16, P16, 1, 16, 28, 4, 128), "GQA_ERR_NULL"),
+    ((P16, P16, P16, ctypes.c_void_p(4), 1, 16, 28, 4, 128), "GQA_ERR_ALIGN"),
+    ((None, None, None, None, 0, 16, 28, 4, 128), "GQA_OK"),
+])
+def test_prefill_rotated_validation(lib, args, code):
+    assert lib.gqa_prefill_rotated(*args) == codes()[code]
+
+
+@pytest.mark.parametrize("args,code", [
+    ((P16, P16, None, P16, -1, 256, 256), "GQA_ERR_DIMS"),
+    ((P16, P16, None, P16, 16, 100, 256), "GQA_ERR_DIMS"),     # d_in not a multiple of 8
+    ((P16, P16, None, P16, 16, 256, 200), "GQA_ERR_DIMS"),     # d_model not a multiple of 128
+    ((None, P16, None, P16, 16, 256, 256), "GQA_ERR_NULL"),
+    ((P16, P16, ctypes.c_void_p(24), P16, 16, 256, 256), "GQA_ERR_ALIGN"),
+    ((None, None, None, None, 0, 256, 256), "GQA_OK"),
+])
+def test_out_proj_validation(lib, args, code):
+    assert lib.gqa_out_proj(*args) == codes()[code]
 
 
 def test_set_stream_accepts_null(lib):

@@ -116,3 +116,51 @@ def test_qkv_then_attention_matches_gqa_prefill_on_the_raw_projection(G):
     out2 = G.prefill(torch.from_numpy(np.ascontiguousarray(q_raw)).to(torch.bfloat16).to(dev), k, v, theta=w.theta)
     assert G.last_error() == 0
     assert_close(out1, out2.float().cpu().numpy(), "rotated route vs prep route")
+
+
+# ---------------------------------------------------------------- output projection + residual
+@pytest.mark.parametrize("T,d_in,dm,resid,inplace", [
+    (200, 256, 256, True, False),    # 2 token tiles, the second ragged
+    (130, 512, 896, True, True),     # 3.5 column tiles (Qwen2-0.5B hidden size), updated in place
+    (64, 72, 128, False, False),     # d_in not a multiple of the 64-wide K block, no residual
+])
+def test_out_proj_small_full_output(G, T, d_in, dm, resid, inplace):
+    rng = torch.Generator().manual_seed(T + d_in + dm)
+    attn = torch.randn(T, d_in, generator=rng).to(torch.bfloat16)
+    w_o = (torch.randn(dm, d_in, generator=rng) / d_in ** 0.5).to(torch.bfloat16)
+    res = torch.randn(T, dm, generator=rng).to(torch.bfloat16) if resid else None
+    dev = torch.device("cuda")
+    res_d = res.to(dev) if resid else None
+    got = G.out_proj(attn.to(dev), w_o.to(dev), res_d, out=res_d if inplace else None)
+    assert G.last_error() == 0
+    assert_rounded(got.float().cpu().numpy(), R.out_proj_ref(attn, w_o, res), f"out_proj T={T} {d_in}->{dm}")
+
+
+def test_out_proj_full_size_sampled_rows(G):
+    w = gi.BY_NAME["qwen2-7b-prefill-L4096"]
+    attn, w_o, res = gi.out_proj_inputs(w)
+    got = G.out_proj(attn.cuda(), w_o.cuda(), res.cuda()).float().cpu().numpy()
+    rows = [0, 1, 127, 128, 2047, 4094, 4095]
+    assert_rounded(got[rows], R.out_proj_ref(attn[rows], w_o, res[rows]), "out_proj Qwen2-7B sampled rows")
+
+
+def test_attention_sublayer_end_to_end(G):
+    """Steps 1-6 of the single-layer data flow on the GPU (projection + RoPE, attention on the rotated
+    inputs, W_O + residual) against the oracles chained the same way."""
+    B, L, h_q, h_kv, d, dm = 1, 300, 28, 4, 128, 512
+    w = gi.small("prefill", B=B, L=L, h_q=h_q, h_kv=h_kv, d=d, seed=77)
+    x, wq, b = gi.qkv_inputs(w, d_model=dm)
+    rng = torch.Generator().manual_seed(78)
+    w_o = (torch.randn(dm, h_q * d, generator=rng) / (h_q * d) ** 0.5).to(torch.bfloat16)
+    x_in = torch.randn(B * L, dm, generator=rng).to(torch.bfloat16)
+    dev = torch.device("cuda")
+    qr, kr, k, v = G.qkv_rope(x.to(dev), wq.to(dev), b.to(dev), h_q, h_kv, theta=w.theta)
+    heads = G.prefill_rotated(qr, kr, v)
+    y = G.out_proj(heads, w_o.to(dev), x_in.to(dev)).float().cpu().numpy()
+    assert G.last_error() == 0
+    qr_r, kr_r, k_r, v_r = R.qkv_rope_ref(x, wq, b, h_q, h_kv, d, w.theta)
+    pos = np.arange(L)
+    q_raw = R.rope(qr_r[0].transpose(1, 0, 2), -pos, w.theta)[None]
+    heads_r = R.prefill_ref(q_raw, k_r, v_r, w.theta)
+    ref = R.out_proj_ref(heads_r.reshape(B * L, h_q * d), w_o, x_in)
+    assert_close(y, ref, "attention sub-layer end to end")
