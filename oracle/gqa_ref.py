@@ -42,11 +42,20 @@ into independent blocks (each block is still the full materialised product):
   7. Output projection and residual (aicoding.csdn.net page, §4.1.3 steps
      5-6): the concatenated heads times W_O, plus the sub-layer input.
      ``out_proj_ref``.
+  8. YaRN scaling of RoPE for contexts beyond the trained window (yudonglee.me
+     page, §6.2: per-dimension interpolation f_i / s * alpha_i with a ramp
+     alpha_i; aicoding.csdn.net page, §5.3: a length-dependent rescaling of
+     the attention logits).  The pages give neither the ramp's bounds nor
+     the rescaling formula; ``Yarn`` takes the published YaRN method's
+     (turn-count bounds 1 and 32, temperature (0.1 ln s + 1)^2): parity
+     partly unpinned.  Pass a ``Yarn`` wherever ``theta`` is taken.
 
 Every function is pinned by ``tests/test_oracle_pins.py`` against closed forms,
 invariants the pages state and a brute-force restatement.
 """
 from __future__ import annotations
+
+from typing import NamedTuple
 
 import numpy as np
 
@@ -63,20 +72,50 @@ def head_group(t: int, g: int) -> int:
     return t // g
 
 
-def inv_freq(d: int, theta: float) -> np.ndarray:
-    """theta^(-2i/d) for i = 0 .. d/2 - 1 (intelliparadigm.com page, §2.3, with d the head size)."""
+class Yarn(NamedTuple):
+    """A RoPE base with YaRN scaling, usable wherever a plain base `theta` is (step 8 of the module
+    docstring).  factor s = 1 is plain RoPE."""
+    base: float
+    factor: float
+    original_max: int
+    beta_fast: float = 32.0
+    beta_slow: float = 1.0
+
+
+def inv_freq(d: int, theta) -> np.ndarray:
+    """theta^(-2i/d) for i = 0 .. d/2 - 1 (intelliparadigm.com page, §2.3, with d the head size).
+
+    With a Yarn spec (yudonglee.me page, §6.2): f'_i = f_i / s * alpha_i, where alpha_i ramps from 1 to s
+    over the dimension pairs: alpha_i = 1 + gamma_i (s - 1), gamma_i = clip((r_i - beta_slow) /
+    (beta_fast - beta_slow), 0, 1), r_i = original_max * f_i / (2 pi) the turns of pair i over the
+    original window.  Pairs that turn many times keep their frequency; slow ones are interpolated by s.
+    """
+    base = theta.base if isinstance(theta, Yarn) else float(theta)
     i = np.arange(d // 2, dtype=np.float64)
-    return np.power(float(theta), -2.0 * i / d)
+    f = np.power(float(base), -2.0 * i / d)
+    if isinstance(theta, Yarn) and theta.factor != 1.0:
+        r = theta.original_max * f / (2.0 * np.pi)
+        gamma = np.clip((r - theta.beta_slow) / (theta.beta_fast - theta.beta_slow), 0.0, 1.0)
+        f = f / theta.factor * (1.0 + gamma * (theta.factor - 1.0))
+    return f
 
 
-def rope(x: np.ndarray, positions, theta: float) -> np.ndarray:
+def rope_mscale(theta) -> float:
+    """YaRN's attention temperature as a factor on the rotated Q and K rows: 0.1 ln(s) + 1, so the scores
+    scale by its square (aicoding.csdn.net page, §5.3: a length-dependent rescaling of the attention
+    logits); 1 without scaling."""
+    return 0.1 * np.log(theta.factor) + 1.0 if isinstance(theta, Yarn) and theta.factor > 1.0 else 1.0
+
+
+def rope(x: np.ndarray, positions, theta) -> np.ndarray:
     """Rotate rows of x [..., P, H, d] at positions [P] (step 1 of the module docstring)."""
     x = np.asarray(x, dtype=np.float64)
     d = x.shape[-1]
     h = d // 2
     ang = np.asarray(positions, dtype=np.float64)[:, None] * inv_freq(d, theta)[None, :]
-    c = np.cos(ang)[:, None, :]
-    s = np.sin(ang)[:, None, :]
+    m = rope_mscale(theta)
+    c = m * np.cos(ang)[:, None, :]
+    s = m * np.sin(ang)[:, None, :]
     x1 = x[..., :h]
     x2 = x[..., h:]
     return np.concatenate([x1 * c - x2 * s, x2 * c + x1 * s], axis=-1)
