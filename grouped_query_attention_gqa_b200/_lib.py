@@ -51,6 +51,8 @@ def load() -> ctypes.CDLL:
     lib.gqa_prefill_rotated.restype = i
     lib.gqa_out_proj.argtypes = [vp, vp, vp, vp, i, i, i]
     lib.gqa_out_proj.restype = i
+    lib.gqa_set_rope_scaling.argtypes = [f, i]
+    lib.gqa_set_rope_scaling.restype = i
     lib.gqa_set_timing_events.argtypes = [vp, vp]
     lib.gqa_set_timing_events.restype = i
     lib.gqa_set_stream.argtypes = [vp]
@@ -243,6 +245,13 @@ def out_proj(attn: torch.Tensor, w_o: torch.Tensor, residual: torch.Tensor | Non
     if rc != GQA_OK:
         raise GQAError(rc, "gqa_out_proj")
     return out
+
+
+def set_rope_scaling(factor: float = 1.0, original_max_position: int = 0) -> None:
+    """YaRN scaling of RoPE (factor s, trained window) for later calls; factor 1 turns it off."""
+    rc = load().gqa_set_rope_scaling(float(factor), int(original_max_position))
+    if rc != GQA_OK:
+        raise GQAError(rc, "gqa_set_rope_scaling")
 
 
 def last_error(device=None) -> int:

@@ -77,7 +77,7 @@ struct Params {
     float* part;               // [(P + B) * h_kv * n_hb * PART]
     int B, h_q, h_kv, g, n_hb, P;
     float scale_log2;
-    double theta;
+    RopeSpec rope;             // RoPE base and YaRN scaling (its temperature is in scale_log2)
     int* err;
 };
 
@@ -208,11 +208,11 @@ __global__ void __launch_bounds__(WARPS * 32, CTAS_PER_SM) split_kernel(const Pa
     const int u = uh / p.n_hb, hb = uh % p.n_hb;
     const int w = gi * WARPS + warp;
 
-    for (int i = threadIdx.x; i < H; i += blockDim.x) finv[i] = rope_inv_freq(i, D, p.theta);
+    for (int i = threadIdx.x; i < H; i += blockDim.x) finv[i] = rope_freq(i, D, p.rope);
     for (int i = threadIdx.x; i < H / 2; i += blockDim.x) {
         float c0, s0, c1, s1;
-        rope_cossin(8.0, rope_inv_freq(2 * i, D, p.theta), c0, s0);
-        rope_cossin(8.0, rope_inv_freq(2 * i + 1, D, p.theta), c1, s1);
+        rope_cossin(8.0, rope_freq(2 * i, D, p.rope), c0, s0);
+        rope_cossin(8.0, rope_freq(2 * i + 1, D, p.rope), c1, s1);
         rot8[i] = make_float4(c0, c1, s0, s1);
     }
     if (lane == 0) {

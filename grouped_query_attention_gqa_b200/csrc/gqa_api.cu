@@ -46,7 +46,8 @@ struct DeviceState {
     void* tab = nullptr;
     size_t tab_bytes = 0;
     int tab_L = -1, tab_d = 0;
-    float tab_theta = 0.f;
+    float tab_theta = 0.f, tab_factor = 1.f;
+    int tab_orig = 0;
     bool qkv_ready[2] = {false, false};
     const void* qkv_key[2] = {nullptr, nullptr};
     long long qkv_dims[3] = {0, 0, 0};
@@ -60,6 +61,17 @@ struct DeviceState {
 DeviceState g_dev[kMaxDevices];
 cudaStream_t g_stream = nullptr;
 cudaEvent_t g_ev_start = nullptr, g_ev_stop = nullptr;   // optional timing of the main kernel
+
+// YaRN scaling of RoPE for every later call (gqa_set_rope_scaling); factor 1 = plain RoPE.
+float g_rope_factor = 1.0f;
+int g_rope_orig = 0;
+
+gqa::RopeSpec rope_spec(float theta) {
+    return gqa::RopeSpec{std::log2(static_cast<double>(theta)), g_rope_factor > 1.0f ? static_cast<double>(g_rope_factor) : 1.0,
+                    static_cast<double>(g_rope_orig)};
+}
+// YaRN's temperature on each rotated row: the logits scale by its square.
+float rope_mscale() { return g_rope_factor > 1.0f ? static_cast<float>(0.1 * std::log(g_rope_factor) + 1.0) : 1.0f; }
 
 inline void mark(cudaEvent_t ev) {
     if (g_ev_start && g_ev_stop) cudaEventRecord(ev, g_stream);
@@ -268,7 +280,7 @@ int launch_prefill(DeviceState* st, const void* q, const void* k, const void* v,
     const int prep_blocks = (L + PREP_POS - 1) / PREP_POS;
     prep_kernel<D><<<prep_blocks, PREP_THREADS, 0, g_stream>>>(static_cast<const __nv_bfloat16*>(q),
                                                                static_cast<const __nv_bfloat16*>(k), qr, kr, B, L,
-                                                               h_q, h_kv, std::log2(static_cast<double>(theta)));
+                                                               h_q, h_kv, rope_spec(theta), rope_mscale());
     if (cudaGetLastError() != cudaSuccess) return GQA_ERR_LAUNCH;
     return launch_attention<D>(st, qr, kr, v, out, B, L, h_q, h_kv, true);
 }
@@ -277,16 +289,20 @@ int launch_prefill(DeviceState* st, const void* q, const void* k, const void* v,
 template <int D>
 int ensure_rope_table(DeviceState* st, int L, float theta) {
     using namespace gqa::qkv;
-    if (st->tab && st->tab_L >= L && st->tab_d == D && st->tab_theta == theta) return GQA_OK;
+    if (st->tab && st->tab_L >= L && st->tab_d == D && st->tab_theta == theta && st->tab_factor == g_rope_factor &&
+        st->tab_orig == g_rope_orig)
+        return GQA_OK;
     const size_t bytes = static_cast<size_t>(L) * (D / 2) * sizeof(float2);
     if (!ensure(st->tab, st->tab_bytes, bytes)) return GQA_ERR_ALLOC;
     const long long n = static_cast<long long>(L) * (D / 2);
     rope_table_kernel<D><<<static_cast<unsigned>((n + TABLE_THREADS - 1) / TABLE_THREADS), TABLE_THREADS, 0,
-                           g_stream>>>(static_cast<float2*>(st->tab), L, std::log2(static_cast<double>(theta)));
+                           g_stream>>>(static_cast<float2*>(st->tab), L, rope_spec(theta), rope_mscale());
     if (cudaGetLastError() != cudaSuccess) return GQA_ERR_LAUNCH;
     st->tab_L = L;
     st->tab_d = D;
     st->tab_theta = theta;
+    st->tab_factor = g_rope_factor;
+    st->tab_orig = g_rope_orig;
     return GQA_OK;
 }
 
@@ -430,7 +446,8 @@ int launch_decode(DeviceState* st, const void* q, const void* kc, const void* vc
     p.n_hb = n_hb;
     p.P = P;
     p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
-    p.theta = static_cast<double>(theta);
+    p.rope = rope_spec(theta);
+    p.scale_log2 *= rope_mscale() * rope_mscale();   // YaRN temperature (1 without scaling)
     p.err = st->err;
 
     plan_kernel<<<1, PLAN_THREADS, 0, g_stream>>>(seqlens, static_cast<int64_t*>(st->dws), B, st->err);
@@ -507,7 +524,8 @@ int launch_decode_fixed_scratch(DeviceState* st, const void* q, const void* kc, 
     p.n_hb = n_hb;
     p.P = P;
     p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
-    p.theta = static_cast<double>(theta);
+    p.rope = rope_spec(theta);
+    p.scale_log2 *= rope_mscale() * rope_mscale();   // YaRN temperature (1 without scaling)
     p.err = st->err;
 
     plan_kernel<<<1, PLAN_THREADS, 0, g_stream>>>(seqlens, static_cast<int64_t*>(st->fixed_scratch), B, st->err);
@@ -548,6 +566,14 @@ const char* gqa_strerror(int code) {
 int gqa_set_timing_events(void* start_event, void* stop_event) {
     g_ev_start = static_cast<cudaEvent_t>(start_event);
     g_ev_stop = static_cast<cudaEvent_t>(stop_event);
+    return GQA_OK;
+}
+
+int gqa_set_rope_scaling(float factor, int original_max_position) {
+    if (!(factor >= 1.0f) || !std::isfinite(factor)) return GQA_ERR_DIMS;
+    if (factor > 1.0f && original_max_position <= 0) return GQA_ERR_DIMS;
+    g_rope_factor = factor;
+    g_rope_orig = factor > 1.0f ? original_max_position : 0;
     return GQA_OK;
 }
 

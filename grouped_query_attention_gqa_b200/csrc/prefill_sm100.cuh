@@ -140,7 +140,7 @@ __global__ void __launch_bounds__(PREP_THREADS, GQA_PREP_MIN_CTAS) prep_kernel(c
                                                             const __nv_bfloat16* __restrict__ k,
                                                             __nv_bfloat16* __restrict__ qr,
                                                             __nv_bfloat16* __restrict__ kr, int B, int L,
-                                                            int h_q, int h_kv, double log2_theta) {
+                                                            int h_q, int h_kv, RopeSpec rope, float mscale) {
     constexpr int H = D / 2;
     constexpr int CH = D / 16;   // one work item = 8 pairs: a 16-byte chunk of the first half + its partner
     // Table row pp holds the D/2 (cos, sin) pairs of position p0 + pp, one padding slot after every 8, so
@@ -189,14 +189,14 @@ __global__ void __launch_bounds__(PREP_THREADS, GQA_PREP_MIN_CTAS) prep_kernel(c
     int base = threadIdx.x;
     load_round(base);
 
-    // theta^(-2i/D) = 2^(-(2i/D) * log2(theta))
-    for (int i = threadIdx.x; i < H; i += blockDim.x) finv[i] = exp2(-(2.0 * i / D) * log2_theta);
+    // theta^(-2i/D) = 2^(-(2i/D) * log2(theta)), scaled under YaRN
+    for (int i = threadIdx.x; i < H; i += blockDim.x) finv[i] = rope_freq(i, D, rope);
     __syncthreads();
     for (int e = threadIdx.x; e < PREP_POS * H; e += blockDim.x) {
         const int pp = e / H, i = e % H;
         float c = 1.f, s = 0.f;
         if (p0 + pp < L) rope_cossin(static_cast<double>(p0 + pp), finv[i], c, s);
-        tab[pp * TROW + i + i / 8] = make_float2(c, s);
+        tab[pp * TROW + i + i / 8] = make_float2(c * mscale, s * mscale);   // YaRN temperature on Q and K
     }
     __syncthreads();
 

@@ -68,18 +68,18 @@ struct alignas(8) Shared {
 };
 
 // ---------------------------------------------------------------------------------------------
-// The cos / sin table: tab[pos * d/2 + i] = (cos, sin)(pos * theta^(-2i/d)), the angle formed in double
-// precision (rope_cossin).
+// The cos / sin table: tab[pos * d/2 + i] = mscale * (cos, sin)(pos * f_i), f_i = rope_freq (theta^(-2i/d),
+// YaRN-scaled if enabled), the angle formed in double precision (rope_cossin).
 template <int D>
 __global__ void __launch_bounds__(TABLE_THREADS) rope_table_kernel(float2* __restrict__ tab, int L,
-                                                                   double log2_theta) {
+                                                                   RopeSpec rope, float mscale) {
     constexpr int H = D / 2;
     const int64_t e = static_cast<int64_t>(blockIdx.x) * TABLE_THREADS + threadIdx.x;
     if (e >= static_cast<int64_t>(L) * H) return;
     const int pos = static_cast<int>(e / H), i = static_cast<int>(e % H);
     float c, s;
-    rope_cossin(static_cast<double>(pos), exp2(-(2.0 * i / D) * log2_theta), c, s);
-    tab[e] = make_float2(c, s);
+    rope_cossin(static_cast<double>(pos), rope_freq(i, D, rope), c, s);
+    tab[e] = make_float2(c * mscale, s * mscale);   // YaRN temperature on Q and K (1 without scaling)
 }
 
 // ---------------------------------------------------------------------------------------------

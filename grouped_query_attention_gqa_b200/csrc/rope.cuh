@@ -24,9 +24,33 @@ constexpr double kTwoPiHi = 6.283185307179586;        // the double nearest 2*pi
 constexpr double kTwoPiLo = 2.4492935982947064e-16;   // 2*pi - kTwoPiHi
 constexpr double kInvTwoPi = 0.15915494309189535;     // 1 / (2*pi), rounded
 
-// theta^(-2i/d)
-__device__ __forceinline__ double rope_inv_freq(int i, int d, double theta) {
-    return pow(theta, -2.0 * static_cast<double>(i) / static_cast<double>(d));
+// YaRN scaling of the frequencies, for contexts beyond the trained window (page "Qwen-2 explained",
+// yudonglee.me, §6.2: f'_i = f_i / s * alpha_i with a per-pair ramp alpha_i from 1 to s; page "Qwen2
+// architecture introduction", aicoding.csdn.net, §5.3: the attention logits are rescaled with the
+// length).  The pages give neither the ramp's bounds nor the rescaling: both follow the published YaRN
+// method.  alpha_i = 1 + gamma_i (s - 1), gamma_i = clamp((r_i - 1) / (32 - 1), 0, 1), where r_i =
+// orig * f_i / (2 pi) is the number of turns pair i makes over the original window: pairs turning 32
+// times or more keep their frequency, pairs turning at most once are interpolated by s.  The logits are
+// scaled by mscale^2, mscale = 0.1 ln(s) + 1 (applied by the callers).  factor <= 1: no scaling.
+constexpr double kYarnTurnsSlow = 1.0;
+constexpr double kYarnTurnsFast = 32.0;
+
+struct RopeSpec {
+    double log2_theta;   // log2 of the RoPE base
+    double factor;       // YaRN factor s (1 = plain RoPE)
+    double orig;         // original (trained) window, in positions
+};
+
+// The (possibly scaled) frequency of pair i: theta^(-2i/d), times alpha_i / s under YaRN.
+__device__ __forceinline__ double rope_freq(int i, int d, const RopeSpec& r) {
+    double f = exp2(-(2.0 * static_cast<double>(i) / static_cast<double>(d)) * r.log2_theta);
+    if (r.factor > 1.0) {
+        const double turns = r.orig * f * kInvTwoPi;
+        double g = (turns - kYarnTurnsSlow) / (kYarnTurnsFast - kYarnTurnsSlow);
+        g = g < 0.0 ? 0.0 : (g > 1.0 ? 1.0 : g);
+        f = f / r.factor * (1.0 + g * (r.factor - 1.0));
+    }
+    return f;
 }
 
 // cos and sin of the angle pos * f.

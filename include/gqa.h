@@ -186,6 +186,23 @@ GQA_API int gqa_prefill_rotated(const void* qr, const void* kr, const void* v, v
 GQA_API int gqa_out_proj(const void* attn, const void* w_o, const void* residual, void* out, int T, int d_in,
                          int d_model);
 
+/*
+ * gqa_set_rope_scaling -- YaRN scaling of RoPE for every later gqa_prefill, gqa_decode, gqa_decode_paged,
+ * gqa_decode_noalloc and gqa_qkv_rope call, for contexts beyond the trained window (page "Qwen-2
+ * explained", yudonglee.me, §6.2: frequencies f_i / s * alpha_i with a per-pair ramp alpha_i; page "Qwen2
+ * architecture introduction", aicoding.csdn.net, §5.3: the attention logits are rescaled).  The pages give
+ * neither the ramp's bounds nor the rescaling; both follow the published YaRN method: alpha_i = 1 +
+ * gamma_i (s - 1) with gamma_i = clamp((r_i - 1) / 31, 0, 1), r_i = original_max_position * f_i / (2 pi),
+ * and the logits multiplied by (0.1 ln s + 1)^2.
+ *   factor                 s >= 1; 1 turns scaling off (the default)
+ *   original_max_position  the trained window (Qwen2: 32768); must be > 0 when factor > 1
+ * The page (aicoding.csdn.net, §5.5) notes the scaled model behaves as the plain one within the trained
+ * window: enabling scaling only for contexts longer than it is left to the caller.  gqa_prefill_rotated
+ * takes Q' and K' as given (gqa_qkv_rope folds the temperature into them).  Process-global, like the
+ * stream; returns GQA_ERR_DIMS for invalid values (the setting is then unchanged).
+ */
+GQA_API int gqa_set_rope_scaling(float factor, int original_max_position);
+
 /* Stream for subsequent calls (a cudaStream_t passed as void*; NULL = legacy stream). */
 GQA_API int gqa_set_stream(void* cuda_stream);
 

@@ -158,5 +158,14 @@ def test_out_proj_validation(lib, args, code):
     assert lib.gqa_out_proj(*args) == codes()[code]
 
 
+@pytest.mark.parametrize("factor,orig,code", [
+    (0.5, 32768, "GQA_ERR_DIMS"), (float("nan"), 32768, "GQA_ERR_DIMS"), (float("inf"), 32768, "GQA_ERR_DIMS"),
+    (4.0, 0, "GQA_ERR_DIMS"), (4.0, 32768, "GQA_OK"), (1.0, 0, "GQA_OK"),
+])
+def test_set_rope_scaling_validation(lib, factor, orig, code):
+    assert lib.gqa_set_rope_scaling(ctypes.c_float(factor), orig) == codes()[code]
+    lib.gqa_set_rope_scaling(ctypes.c_float(1.0), 0)
+
+
 def test_set_stream_accepts_null(lib):
     assert lib.gqa_set_stream(None) == 0
