@@ -48,13 +48,12 @@ struct DeviceState {
     int tab_L = -1, tab_d = 0;
     float tab_theta = 0.f, tab_factor = 1.f;
     int tab_orig = 0;
-    bool qkv_ready[2] = {false, false};
+    unsigned gemm_ready = 0;   // bit per GEMM kernel instantiation whose shared-memory size is set
     const void* qkv_key[2] = {nullptr, nullptr};
-    long long qkv_dims[3] = {0, 0, 0};
+    long long qkv_dims[4] = {0, 0, 0, 0};
     CUtensorMap qkv_maps[2];
-    bool proj_ready = false;
     const void* proj_key[2] = {nullptr, nullptr};
-    long long proj_dims[3] = {0, 0, 0};
+    long long proj_dims[4] = {0, 0, 0, 0};
     CUtensorMap proj_maps[2];
 };
 
@@ -306,6 +305,47 @@ int ensure_rope_table(DeviceState* st, int L, float theta) {
     return GQA_OK;
 }
 
+// X [T, K] and W [N, K] tensor maps of a projection GEMM with tile width bn, reused while the key matches.
+bool gemm_maps(CUtensorMap* maps, const void** key, long long* dims, const void* x, const void* w, long long T,
+               int K, long long N, int bn) {
+    using namespace gqa::qkv;
+    if (key[0] == x && key[1] == w && dims[0] == T && dims[1] == N && dims[2] == K && dims[3] == bn) return true;
+    key[0] = key[1] = nullptr;
+    if (!get_encoder()) return false;
+    const cuuint64_t sx[1] = {static_cast<cuuint64_t>(K) * 2};
+    const cuuint64_t dx[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(T)};
+    const cuuint32_t bx[2] = {BK, BM};
+    if (!encode_bf16(&maps[0], const_cast<void*>(x), 2, dx, sx, bx)) return false;
+    const cuuint64_t dw[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(N)};
+    const cuuint32_t bw[2] = {BK, static_cast<cuuint32_t>(bn)};
+    if (!encode_bf16(&maps[1], const_cast<void*>(w), 2, dw, sx, bw)) return false;
+    key[0] = x;
+    key[1] = w;
+    dims[0] = T;
+    dims[1] = N;
+    dims[2] = K;
+    dims[3] = bn;
+    return true;
+}
+
+// Launch one instantiation of the persistent GEMM (the kernel `fn`, tile width BN) over p.n_tiles tiles.
+template <int BN>
+int run_gemm(DeviceState* st, void (*fn)(CUtensorMap, CUtensorMap, gqa::qkv::Params), unsigned ready_bit,
+             const CUtensorMap* maps, const gqa::qkv::Params& p) {
+    using namespace gqa::qkv;
+    if (!(st->gemm_ready & ready_bit)) {
+        if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, Tile<BN>::DYN) != cudaSuccess)
+            return GQA_ERR_LAUNCH;
+        st->gemm_ready |= ready_bit;
+    }
+    const int grid = p.n_tiles < st->num_sms ? p.n_tiles : st->num_sms;
+    mark(g_ev_start);
+    fn<<<grid, NUM_THREADS, Tile<BN>::DYN, g_stream>>>(maps[0], maps[1], p);
+    if (cudaGetLastError() != cudaSuccess) return GQA_ERR_LAUNCH;
+    mark(g_ev_stop);
+    return GQA_OK;
+}
+
 template <int D>
 int launch_qkv(DeviceState* st, const void* x, const void* w, const void* bias, void* qr, void* kr, void* k,
                void* v, int B, int L, int d_model, int h_q, int h_kv, float theta) {
@@ -314,26 +354,10 @@ int launch_qkv(DeviceState* st, const void* x, const void* w, const void* bias, 
     if (rc != GQA_OK) return rc;
     const long long T = static_cast<long long>(B) * L;
     const int N = (h_q + 2 * h_kv) * D;
-    if (!get_encoder()) return GQA_ERR_LAUNCH;
-    if (st->qkv_key[0] != x || st->qkv_key[1] != w || st->qkv_dims[0] != T || st->qkv_dims[1] != N ||
-        st->qkv_dims[2] != d_model) {
-        st->qkv_key[0] = st->qkv_key[1] = nullptr;
-        const cuuint64_t dx[2] = {static_cast<cuuint64_t>(d_model), static_cast<cuuint64_t>(T)};
-        const cuuint64_t sx[1] = {static_cast<cuuint64_t>(d_model) * 2};
-        const cuuint32_t bx[2] = {BK, BM};
-        if (!encode_bf16(&st->qkv_maps[0], const_cast<void*>(x), 2, dx, sx, bx)) return GQA_ERR_LAUNCH;
-        const cuuint64_t dw[2] = {static_cast<cuuint64_t>(d_model), static_cast<cuuint64_t>(N)};
-        const cuuint32_t bw[2] = {BK, BN};
-        if (!encode_bf16(&st->qkv_maps[1], const_cast<void*>(w), 2, dw, sx, bw)) return GQA_ERR_LAUNCH;
-        st->qkv_key[0] = x;
-        st->qkv_key[1] = w;
-        st->qkv_dims[0] = T;
-        st->qkv_dims[1] = N;
-        st->qkv_dims[2] = d_model;
-    }
-    Params p;
-    p.resid = nullptr;
-    p.out = nullptr;
+    const long long mtiles = (T + BM - 1) / BM;
+    constexpr int bn = 256;
+    if (!gemm_maps(st->qkv_maps, st->qkv_key, st->qkv_dims, x, w, T, d_model, N, bn)) return GQA_ERR_LAUNCH;
+    Params p = {};
     p.bias = static_cast<const __nv_bfloat16*>(bias);
     p.tab = static_cast<const float2*>(st->tab);
     p.qr = static_cast<__nv_bfloat16*>(qr);
@@ -345,70 +369,34 @@ int launch_qkv(DeviceState* st, const void* x, const void* w, const void* bias, 
     p.N = N;
     p.h_q = h_q;
     p.h_kv = h_kv;
-    p.n_ntiles = (N + BN - 1) / BN;
-    const long long mtiles = (T + BM - 1) / BM;
+    p.n_ntiles = (N + bn - 1) / bn;
     if (mtiles * p.n_ntiles > 0x7fffffffLL) return GQA_ERR_DIMS;
     p.n_tiles = static_cast<int>(mtiles * p.n_ntiles);
     p.kblocks = (d_model + BK - 1) / BK;
     p.err = st->err;
-    bool& ready = st->qkv_ready[D == 128 ? 1 : 0];
-    if (!ready) {
-        if (cudaFuncSetAttribute(qkv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, DYN) != cudaSuccess)
-            return GQA_ERR_LAUNCH;
-        ready = true;
-    }
-    const int grid = p.n_tiles < st->num_sms ? p.n_tiles : st->num_sms;
-    mark(g_ev_start);
-    qkv_kernel<D><<<grid, NUM_THREADS, DYN, g_stream>>>(st->qkv_maps[0], st->qkv_maps[1], p);
-    if (cudaGetLastError() != cudaSuccess) return GQA_ERR_LAUNCH;
-    mark(g_ev_stop);
-    return GQA_OK;
+    return run_gemm<bn>(st, qkv_kernel<D, bn>, D == 128 ? 1u : 2u, st->qkv_maps, p);
 }
 
 // Output projection + residual: out [T, d_model] = attn [T, d_in] w_o [d_model, d_in]^T (+ resid).
 int launch_proj(DeviceState* st, const void* attn, const void* w_o, const void* resid, void* out, int T, int d_in,
                 int d_model) {
     using namespace gqa::qkv;
-    if (!get_encoder()) return GQA_ERR_LAUNCH;
-    if (st->proj_key[0] != attn || st->proj_key[1] != w_o || st->proj_dims[0] != T || st->proj_dims[1] != d_in ||
-        st->proj_dims[2] != d_model) {
-        st->proj_key[0] = st->proj_key[1] = nullptr;
-        const cuuint64_t sx[1] = {static_cast<cuuint64_t>(d_in) * 2};
-        const cuuint64_t da[2] = {static_cast<cuuint64_t>(d_in), static_cast<cuuint64_t>(T)};
-        const cuuint32_t ba[2] = {BK, BM};
-        if (!encode_bf16(&st->proj_maps[0], const_cast<void*>(attn), 2, da, sx, ba)) return GQA_ERR_LAUNCH;
-        const cuuint64_t dw[2] = {static_cast<cuuint64_t>(d_in), static_cast<cuuint64_t>(d_model)};
-        const cuuint32_t bw[2] = {BK, BN};
-        if (!encode_bf16(&st->proj_maps[1], const_cast<void*>(w_o), 2, dw, sx, bw)) return GQA_ERR_LAUNCH;
-        st->proj_key[0] = attn;
-        st->proj_key[1] = w_o;
-        st->proj_dims[0] = T;
-        st->proj_dims[1] = d_in;
-        st->proj_dims[2] = d_model;
-    }
+    const long long mtiles = (static_cast<long long>(T) + BM - 1) / BM;
+    constexpr int bn = 256;
+    if (!gemm_maps(st->proj_maps, st->proj_key, st->proj_dims, attn, w_o, T, d_in, d_model, bn))
+        return GQA_ERR_LAUNCH;
     Params p = {};
     p.resid = static_cast<const __nv_bfloat16*>(resid);
     p.out = static_cast<__nv_bfloat16*>(out);
     p.T = T;
     p.L = T;
     p.N = d_model;
-    p.n_ntiles = (d_model + BN - 1) / BN;
-    const long long mtiles = (static_cast<long long>(T) + BM - 1) / BM;
+    p.n_ntiles = (d_model + bn - 1) / bn;
     if (mtiles * p.n_ntiles > 0x7fffffffLL) return GQA_ERR_DIMS;
     p.n_tiles = static_cast<int>(mtiles * p.n_ntiles);
     p.kblocks = (d_in + BK - 1) / BK;
     p.err = st->err;
-    if (!st->proj_ready) {
-        if (cudaFuncSetAttribute(proj_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, DYN) != cudaSuccess)
-            return GQA_ERR_LAUNCH;
-        st->proj_ready = true;
-    }
-    const int grid = p.n_tiles < st->num_sms ? p.n_tiles : st->num_sms;
-    mark(g_ev_start);
-    proj_kernel<<<grid, NUM_THREADS, DYN, g_stream>>>(st->proj_maps[0], st->proj_maps[1], p);
-    if (cudaGetLastError() != cudaSuccess) return GQA_ERR_LAUNCH;
-    mark(g_ev_stop);
-    return GQA_OK;
+    return run_gemm<bn>(st, proj_kernel<bn>, 4u, st->proj_maps, p);
 }
 
 // Packed cache (bt == nullptr) or paged cache through the block table bt [B, max_pages].

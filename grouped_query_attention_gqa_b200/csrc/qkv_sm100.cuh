@@ -31,19 +31,30 @@ namespace qkv {
 using namespace ptx;
 
 constexpr int BM = 128;                  // tokens per tile (MMA M, TMEM lanes)
-constexpr int BN = 256;                  // output columns per tile (MMA N)
 constexpr int BK = 64;                   // K block: one 128-byte swizzle atom of bf16
-constexpr int STAGES = 4;
 constexpr int NUM_THREADS = 192;
 constexpr int WARP_TMA = 0, WARP_MMA = 1;
 constexpr int A_BYTES = BM * BK * 2;     // 16 KB
-constexpr int B_BYTES = BN * BK * 2;     // 32 KB
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int EPI_WARPS = 4;
 constexpr int STAGING = 32 * 128 * 2;    // one epilogue warp's 32 rows of up to 128 bf16
-constexpr int DYN = STAGES * STAGE_BYTES + EPI_WARPS * STAGING + 1024;
-constexpr int TMEM_COLS = 2 * BN;
+constexpr int RING_BYTES = 192 * 1024;   // the K-block ring
+constexpr int MAX_STAGES = 6;
 constexpr int TABLE_THREADS = 256;
+
+// Tile width BN (MMA N).  256 columns (a 4-stage ring) is what the kernels are launched with: measured
+// on the Qwen2-7B projections, 128-column tiles (a 6-stage ring) were slower even where they would fill
+// the last wave of CTAs better -- twice the K-block traffic per FLOP and a shorter main loop to hide each
+// epilogue behind.
+template <int BN_>
+struct Tile {
+    static constexpr int BN = BN_;
+    static constexpr int B_BYTES = BN * BK * 2;
+    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+    static constexpr int STAGES = RING_BYTES / STAGE_BYTES;
+    static constexpr int DYN = STAGES * STAGE_BYTES + EPI_WARPS * STAGING + 1024;
+    static constexpr int TMEM_COLS = 2 * BN;   // two accumulators
+    static_assert(STAGES <= MAX_STAGES, "ring deeper than the barrier arrays");
+};
 
 struct Params {
     const __nv_bfloat16* bias;   // [N] or nullptr
@@ -60,7 +71,7 @@ struct Params {
 };
 
 struct alignas(8) Shared {
-    uint64_t full[STAGES], empty[STAGES];
+    uint64_t full[MAX_STAGES], empty[MAX_STAGES];
     uint64_t acc_full[2], acc_empty[2];
     uint64_t mma_done;
     uint32_t tmem_base;
@@ -177,23 +188,41 @@ __device__ __forceinline__ void store_head(const Params& p, float (&y)[D], int n
     }
 }
 
+// The reverse of store_rows: the warp's 32 rows (src per lane, nullptr for none) are read whole rows per
+// load instruction into the staging buffer, then each lane adds its own row to z.
+template <int D>
+__device__ __forceinline__ void add_rows(uint8_t* stage, const __nv_bfloat16* src, float* z, int lane) {
+    constexpr int CH = D / 8;
+    constexpr int RPI = 32 / CH;
+    uint4* st = reinterpret_cast<uint4*>(stage);
+    const uint64_t mine = reinterpret_cast<uint64_t>(src);
+    const int c = lane % CH;
+#pragma unroll
+    for (int j = 0; j < 32 / RPI; ++j) {
+        const int r = j * RPI + lane / CH;
+        const uint64_t row = __shfl_sync(0xffffffffu, mine, r);
+        st[r * CH + (c ^ (r & (CH - 1)))] = row ? reinterpret_cast<const uint4*>(row)[c] : make_uint4(0, 0, 0, 0);
+    }
+    __syncwarp();
+#pragma unroll
+    for (int cc = 0; cc < CH; ++cc) {
+        const uint4 w = st[lane * CH + (cc ^ (lane & (CH - 1)))];
+        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            z[8 * cc + 2 * e] += bf16lo_to_f32(ws[e]);
+            z[8 * cc + 2 * e + 1] += bf16hi_to_f32(ws[e]);
+        }
+    }
+    __syncwarp();   // the buffer is reused by the next call
+}
+
 // The output projection's epilogue: 128 columns of one row per lane, + the residual, stored as rows.
 __device__ __forceinline__ void store_resid(const Params& p, float (&y)[128], int n0, int t, bool valid,
                                             uint8_t* stage, int lane) {
-    if (p.resid && valid) {
-        const uint4* rr = reinterpret_cast<const uint4*>(p.resid + static_cast<int64_t>(t) * p.N + n0);
-#pragma unroll
-        for (int c = 0; c < 16; ++c) {
-            const uint4 w = rr[c];
-            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                y[8 * c + 2 * e] += bf16lo_to_f32(ws[e]);
-                y[8 * c + 2 * e + 1] += bf16hi_to_f32(ws[e]);
-            }
-        }
-    }
-    store_rows<128>(stage, valid ? p.out + static_cast<int64_t>(t) * p.N + n0 : nullptr, y, lane);
+    const int64_t at = static_cast<int64_t>(t) * p.N + n0;
+    if (p.resid) add_rows<128>(stage, valid ? p.resid + at : nullptr, y, lane);
+    store_rows<128>(stage, valid ? p.out + at : nullptr, y, lane);
 }
 
 enum Epilogue { kQKV = 0, kResidual = 1 };
@@ -201,8 +230,12 @@ enum Epilogue { kQKV = 0, kResidual = 1 };
 // ---------------------------------------------------------------------------------------------
 // The persistent GEMM: Y[T, N] = X[T, K] W[N, K]^T with the epilogue EPI.  For kQKV, D is the head size
 // (tiles are processed head by head); for kResidual, D = 128 (tiles are processed 128 columns at a time).
-template <int D, int EPI>
+template <int D, int EPI, int BN_>
 __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtensorMap& tm_w, const Params& p) {
+    constexpr int BN = Tile<BN_>::BN;
+    constexpr int STAGES = Tile<BN_>::STAGES;
+    constexpr int STAGE_BYTES = Tile<BN_>::STAGE_BYTES;
+    constexpr int TMEM_COLS = Tile<BN_>::TMEM_COLS;
     extern __shared__ uint8_t dyn_smem_raw[];
     __shared__ Shared sh;
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dyn_smem_raw) + 1023) & ~uintptr_t(1023));
@@ -340,17 +373,18 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtenso
     }
 }
 
-template <int D>
+template <int D, int BN>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     qkv_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w, const Params p) {
-    gemm_body<D, kQKV>(tm_x, tm_w, p);
+    gemm_body<D, kQKV, BN>(tm_x, tm_w, p);
 }
 
 // Output projection + residual (page "Qwen2 architecture introduction", §4.1.3 steps 5-6):
 // out = attn W_O + X_in, with attn the concatenated heads [T, h_q d] and W_O^T [d_model, h_q d].
+template <int BN>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     proj_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w, const Params p) {
-    gemm_body<128, kResidual>(tm_x, tm_w, p);
+    gemm_body<128, kResidual, BN>(tm_x, tm_w, p);
 }
 
 }  // namespace qkv

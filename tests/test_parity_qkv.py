@@ -123,6 +123,7 @@ def test_qkv_then_attention_matches_gqa_prefill_on_the_raw_projection(G):
     (200, 256, 256, True, False),    # 2 token tiles, the second ragged
     (130, 512, 896, True, True),     # 3.5 column tiles (Qwen2-0.5B hidden size), updated in place
     (64, 72, 128, False, False),     # d_in not a multiple of the 64-wide K block, no residual
+    (4736, 512, 1024, True, False),  # 37 x 4 tiles: exactly one full wave of 148 CTAs
 ])
 def test_out_proj_small_full_output(G, T, d_in, dm, resid, inplace):
     rng = torch.Generator().manual_seed(T + d_in + dm)
