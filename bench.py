@@ -72,6 +72,8 @@ def load_peaks():
 
 KERNEL_SOURCES = {
     "attn_kernel": ["prefill_sm100.cuh", "sm100_ptx.cuh", "rope.cuh"],
+    "qkv_kernel": ["qkv_sm100.cuh", "sm100_ptx.cuh", "rope.cuh"],
+    "proj_kernel": ["qkv_sm100.cuh", "sm100_ptx.cuh"],
     "split_kernel": ["decode_sm100.cuh", "sm100_ptx.cuh", "rope.cuh"],
 }
 
@@ -414,9 +416,8 @@ def run_ours(args):
     sampler = ClockSampler(local)
     with sampler:
         t_wall = time.perf_counter()
-        for i in range(K):
+        for i in range(K):   # interleaved, so both kinds of step see the same clocks and temperature
             step(evs[i])
-        for i in range(K):
             step(kevs[i], inner=True)
         torch.cuda.synchronize()
         t_wall = time.perf_counter() - t_wall
@@ -478,6 +479,74 @@ def run_ours(args):
         e2e_pre = reduce_max(sum(e[0].elapsed_time(e[1]) for e in e2e_evs) / K, dev)
         e2e_dec = reduce_max(sum(e[1].elapsed_time(e[2]) for e in e2e_evs) / K, dev)
 
+    # ---- the fused route from hidden states: QKV projection + bias + RoPE (writing Q', K' and the cache
+    # rows K, V), then the attention on the rotated inputs -- no prep pass.  Timed like the headline
+    # steps, plus K steps with events around the projection kernel alone.
+    qkv_line = None
+    if do_p and not args.no_qkv:
+        dm = gi.D_MODEL[(wp.h_q, wp.h_kv, wp.d)]
+        xq, wqkv, bqkv = gi.qkv_inputs(wp, d_model=dm, device=str(dev))
+        _, w_o, x_in = gi.out_proj_inputs(wp, d_model=dm, device=str(dev))
+        y_out = torch.empty_like(x_in)
+        qo = (q.new_empty(wp.B, wp.h_q, wp.L, wp.d), q.new_empty(wp.B, wp.h_kv, wp.L, wp.d),
+              q.new_empty(wp.B, wp.L, wp.h_kv, wp.d), q.new_empty(wp.B, wp.L, wp.h_kv, wp.d))
+
+        def qstep(e, inner=False):
+            flush.zero_()
+            e[0].record()
+            if inner:
+                G.set_timing_events(e[1], e[2])
+            G.qkv_rope(xq, wqkv, bqkv, wp.h_q, wp.h_kv, theta=wp.theta, out=qo)
+            if inner:
+                G.set_timing_events(None, None)
+            G.prefill_rotated(qo[0], qo[1], qo[3], out=out)
+            if inner:
+                G.set_timing_events(e[4], e[5])
+            G.out_proj(out, w_o, x_in, out=y_out)
+            if inner:
+                G.set_timing_events(None, None)
+            e[3].record()
+
+        for _ in range(W):
+            qstep([ev() for _ in range(6)])
+        qe = [[ev() for _ in range(6)] for _ in range(K)]
+        qke = [[ev() for _ in range(6)] for _ in range(K)]
+        torch.cuda.synchronize()
+        barrier()
+        for i in range(K):
+            qstep(qe[i])
+            qstep(qke[i], inner=True)
+        torch.cuda.synchronize()
+        barrier()
+        if G.last_error() != 0:
+            raise RuntimeError("device error in the QKV leg")
+        qfl = 2.0 * wp.B * wp.L * dm * (wp.h_q + 2 * wp.h_kv) * wp.d
+        ofl = 2.0 * wp.B * wp.L * (wp.h_q * wp.d) * dm
+        route_ms = reduce_max(sum(e[0].elapsed_time(e[3]) for e in qe) / K, dev)
+        qkv_ms = sum(e[1].elapsed_time(e[2]) for e in qke) / K
+        proj_ms = sum(e[4].elapsed_time(e[5]) for e in qke) / K
+        peaks_q, src_q = load_peaks()
+        qkv_line = {
+            "workload": f"{wp.desc}, d_model={dm}: X [{wp.B * wp.L}, {dm}] x W_qkv^T [{dm}, {(wp.h_q + 2 * wp.h_kv) * wp.d}]"
+                        " + bias, RoPE on Q and K, Q'/K' head-major and K/V cache rows written",
+            "flops_per_step": qfl,
+            "roofline": {"kernel": "qkv_kernel", "bound": "tensor", "achieved": qfl / (qkv_ms * 1e-3) / 1e12,
+                         "peak": peaks_q["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": qfl / (qkv_ms * 1e-3) / 1e12 / peaks_q["bf16_tflops"],
+                         "peak_source": f"{src_q} bf16 dense (burst)",
+                         "traffic": profile_traffic("qkv_kernel", wp.name),
+                         "algorithmic_flops_per_launch": qfl, "ms_per_launch": qkv_ms},
+            "out_proj": {"kernel": "proj_kernel", "bound": "tensor", "flops_per_launch": ofl,
+                         "ms_per_launch": proj_ms, "achieved": ofl / (proj_ms * 1e-3) / 1e12,
+                         "frac": ofl / (proj_ms * 1e-3) / 1e12 / peaks_q["bf16_tflops"], "unit": "TFLOP/s",
+                         "note": "attn [T, h_q d] x W_O^T [h_q d, d_model] + residual"},
+            "sublayer": {"ms_per_step": route_ms,
+                         "value": world * (qfl + fl + ofl) / (route_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                         "note": "the attention sub-layer from hidden states: QKV projection + bias + RoPE, "
+                                 "attention on the rotated inputs, W_O + residual (no prep pass)"},
+        }
+        del xq, wqkv, bqkv, qo, w_o, x_in, y_out
+
     peaks, peak_src = load_peaks()
     kvb = decode_kv_bytes(total_rows, wd)
     allb = decode_bytes(total_rows, wd)
@@ -494,8 +563,8 @@ def run_ours(args):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic: seeded N(0,1) bf16 Q/K/V and caches drawn on the device; decode lengths U[1,32768]",
             "config": dict(bench_config(wp, wd),
-                           timing=f"{K} headline steps without per-kernel events, then {K} steps with CUDA "
-                                  "events around the attention / split kernels for the roofline"),
+                           timing=f"{K} headline steps without per-kernel events, interleaved with {K} steps "
+                                  "with CUDA events around the attention / split kernels for the roofline"),
             "roofline": {"kernel": "attn_kernel (prefill)", "bound": "tensor", "achieved": achieved_t,
                          "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved_t / peaks["bf16_tflops"],
                          "peak_source": f"{peak_src} bf16 dense (burst)",
@@ -506,7 +575,8 @@ def run_ours(args):
             "e2e": {"value": world * fl / (e2e_pre * 1e-3) / 1e12, "unit": "TFLOP/s",
                     "h2d_bytes_per_step": sum(x.numel() * x.element_size() for x in (q, k, v)),
                     "d2h_bytes_per_step": out.numel() * out.element_size()},
-            "gpu_launches": (2 * do_p + 3 * do_d) * 2 * K,
+            "gpu_launches": (2 * do_p + 3 * do_d) * 2 * K + (6 * K if qkv_line else 0),
+            "qkv": qkv_line,
             "clocks": sampler.summary(),
             "decode": {
                 "workload": wd.desc, "total_cache_rows": total_rows,
@@ -553,6 +623,7 @@ def main(argv=None):
                     help="run one half of the step only (profiling; the line then carries that half)")
     ap.add_argument("--prefill-workload", default=PREFILL_WORKLOAD, choices=[w.name for w in gi.WORKLOADS if w.kind == "prefill"],
                     help="prefill workload of the step (default: the Qwen2-7B L=4096 headline workload)")
+    ap.add_argument("--no-qkv", action="store_true", help="skip the fused QKV projection leg")
     ap.add_argument("--decode-page-size", type=int, default=None,
                     help="decode through gqa_decode_paged, the cache in pages of this many rows")
     ap.add_argument("--decode-batch", type=int, default=None,
