@@ -537,6 +537,8 @@ def run_ours(args):
                          "traffic": profile_traffic("qkv_kernel", wp.name),
                          "algorithmic_flops_per_launch": qfl, "ms_per_launch": qkv_ms},
             "out_proj": {"kernel": "proj_kernel", "bound": "tensor", "flops_per_launch": ofl,
+                         "traffic": profile_traffic("proj_kernel", wp.name),
+                         "peak": peaks_q["bf16_tflops"], "peak_source": f"{src_q} bf16 dense (burst)",
                          "ms_per_launch": proj_ms, "achieved": ofl / (proj_ms * 1e-3) / 1e12,
                          "frac": ofl / (proj_ms * 1e-3) / 1e12 / peaks_q["bf16_tflops"], "unit": "TFLOP/s",
                          "note": "attn [T, h_q d] x W_O^T [h_q d, d_model] + residual"},
