@@ -51,6 +51,8 @@ CASES = [
     (1, 64, 72, 2, 1, 128, False),       # d_model not a multiple of the 64-wide K block, no bias
     (3, 97, 896, 14, 2, 64, True),       # Qwen2-0.5B hidden size and heads
     (1, 300, 1024, 8, 8, 128, True),     # MHA (h_q = h_kv)
+    (1, 1152, 256, 28, 4, 128, True),    # 162 tiles: one whole wave of 148 CTAs and 14 more
+    (4, 1024, 512, 14, 2, 64, True),     # d = 64, 160 tiles over 4 sequences
 ]
 
 
@@ -124,6 +126,7 @@ def test_qkv_then_attention_matches_gqa_prefill_on_the_raw_projection(G):
     (130, 512, 896, True, True),     # 3.5 column tiles (Qwen2-0.5B hidden size), updated in place
     (64, 72, 128, False, False),     # d_in not a multiple of the 64-wide K block, no residual
     (4736, 512, 1024, True, False),  # 37 x 4 tiles: exactly one full wave of 148 CTAs
+    (1280, 512, 4096, True, True),   # 160 tiles: one whole wave and 12 more, in place
 ])
 def test_out_proj_small_full_output(G, T, d_in, dm, resid, inplace):
     rng = torch.Generator().manual_seed(T + d_in + dm)
