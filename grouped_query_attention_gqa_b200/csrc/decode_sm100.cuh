@@ -231,7 +231,8 @@ __global__ void __launch_bounds__(WARPS * 32, CTAS_PER_SM) split_kernel(const Pa
     const int t4 = lane >> 2, tq = lane & 3;
     const size_t row_stride = static_cast<size_t>(p.h_kv) * D;
 
-    // ---- producer side of the warp's ring
+    // ---- producer side of the warp's ring.  Every cache row is read once: evict-first in L2.
+    const uint64_t stream_policy = l2_evict_first_policy();
     BlockCursor iss;
     iss.init(p.off, p.B, start, end);
     auto issue = [&](int stage) {
@@ -263,7 +264,7 @@ __global__ void __launch_bounds__(WARPS * 32, CTAS_PER_SM) split_kernel(const Pa
         fence_proxy_async_smem();
         if (load) {
             const __nv_bfloat16* src = (is_v ? p.vc : p.kc) + srow * row_stride + static_cast<size_t>(u) * D;
-            bulk_load(dst, src, D * 2, bar);
+            bulk_load_hint(dst, src, D * 2, bar, stream_policy);
         } else {
 #pragma unroll
             for (int c = 0; c < D / 8; ++c) reinterpret_cast<uint4*>(dst)[c] = make_uint4(0, 0, 0, 0);
