@@ -45,6 +45,7 @@ PREFILL_WORKLOAD = "qwen2-7b-prefill-L4096"
 DECODE_WORKLOAD = "qwen2-7b-decode-B64"
 FLUSH_BYTES = 256 << 20
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+SPEC_BF16_TFLOPS = 2250.0   # dense bf16 of one B200, data sheet (context only)
 
 
 # ------------------------------------------------------------------------------------------ helpers
@@ -433,6 +434,8 @@ def run_ours(args):
     fl = prefill_flops(wp)
     value_tflops = whole_job_rate(fl, 1e-3 * sum(pre_ms) / K, dev) / 1e12   # every rank: same collectives
     pre_mean = reduce_max(sum(pre_ms) / K, dev)
+    if not do_p:   # --only decode: no prefill was timed, so there is no headline value
+        value_tflops = pre_mean = None
     dec_mean = reduce_max(sum(dec_ms) / K, dev)
     attn_mean = sum(attn_ms) / K
     split_mean = sum(split_ms) / K
@@ -554,7 +557,7 @@ def run_ours(args):
     allb = decode_bytes(total_rows, wd)
     line = None
     if rank == 0:
-        achieved_t = fl / (attn_mean * 1e-3) / 1e12
+        achieved_t = fl / (attn_mean * 1e-3) / 1e12 if do_p else None
         achieved_b = allb / (split_mean * 1e-3) / 1e9
         line = {
             "metric": METRIC,
@@ -571,7 +574,13 @@ def run_ours(args):
                          "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved_t / peaks["bf16_tflops"],
                          "peak_source": f"{peak_src} bf16 dense (burst)",
                          "traffic": profile_traffic("attn_kernel", wp.name),
-                         "algorithmic_flops_per_launch": fl, "ms_per_launch": attn_mean},
+                         "algorithmic_flops_per_launch": fl, "ms_per_launch": attn_mean,
+                         # beside the burst peak: the sustained cuBLAS figure and the 2.25 PFLOP/s data-sheet
+                         # number, and the exponentials per launch (one per unmasked score)
+                         "frac_of_sustained": achieved_t / peaks["bf16_tflops_sustained"],
+                         "frac_of_spec": achieved_t / SPEC_BF16_TFLOPS,
+                         "exp_per_launch": wp.B * wp.h_q * wp.L * (wp.L + 1) // 2,
+                         "exp_per_s": wp.B * wp.h_q * wp.L * (wp.L + 1) / 2 / (attn_mean * 1e-3)},
             "cpu_baseline": cpu_baseline(wp) if (world == 1 and not args.no_cpu_baseline) else None,
             "only": args.only,
             "e2e": {"value": world * fl / (e2e_pre * 1e-3) / 1e12, "unit": "TFLOP/s",
@@ -601,6 +610,10 @@ def run_ours(args):
             "wall_s_timed_region": t_wall,
             "impl": "ours",
         }
+        if not do_p:   # --only decode: the line carries the decode half alone
+            line["roofline"] = line["e2e"] = line["cpu_baseline"] = None
+        if not do_d:   # --only prefill
+            line["decode"] = None
     if torch.distributed.is_initialized():
         barrier()
         torch.distributed.destroy_process_group()

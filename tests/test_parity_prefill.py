@@ -77,6 +77,43 @@ def test_prefill_theta_1e4_and_repeat_calls(G):
         assert_close(run(G, q, k, v, w.theta), ref, "theta=1e4")
 
 
+def spike_inputs(B, L, h_q, h_kv, d, seed, step_log2=9.5, alpha=4.0):
+    """Inputs whose running row maximum grows by more than 2^8 from one key tile to the next.
+
+    Q and K are small noise plus a component along the pair of dimensions RoPE turns slowest (d/2-1 and
+    d-1; at theta = 1e6 it turns by ~1e-6 rad per position, so the rotation leaves that part of the logits
+    unchanged).  Key 128t + 5 of every tile t >= 1 carries a spike whose logit is step_log2 * t in log2
+    units; all other logits stay near 0.  A row of query tile 1 thus weighs its 128 + 127 plain keys
+    against one spike ~2^9.5 times heavier: the lazy rescale of the running output has to happen, and the
+    plain keys still make ~15 % of the result, so a wrong rescale shows.
+    """
+    gen = torch.Generator().manual_seed(seed)
+    q = 0.3 * torch.randn(B, L, h_q, d, generator=gen)
+    k = 0.3 * torch.randn(B, L, h_kv, d, generator=gen)
+    v = torch.randn(B, L, h_kv, d, generator=gen)
+    slow = [d // 2 - 1, d - 1]
+    q[..., slow] += alpha
+    beta = step_log2 * np.log(2.0) * np.sqrt(d) / (2 * alpha)   # spike component per tile step
+    for t in range(1, (L + 127) // 128):
+        if 128 * t + 5 < L:
+            k[:, 128 * t + 5, :, slow] += beta * t
+    return q.to(torch.bfloat16), k.to(torch.bfloat16), v.to(torch.bfloat16)
+
+
+@pytest.mark.parametrize("B,L,h_q,h_kv,d", [(1, 700, 28, 4, 128), (2, 400, 8, 2, 64)])
+def test_prefill_running_max_grows_across_key_tiles(G, B, L, h_q, h_kv, d):
+    q, k, v = spike_inputs(B, L, h_q, h_kv, d, seed=L + d)
+    # The construction does what it says: unrotated logits (the rotation moves them by < 1e-3 here) of the
+    # spikes step up by more than 8 log2 units per key tile.
+    qf, kf = q.float().numpy(), k.float().numpy()
+    lg = np.einsum("d,d->", qf[0, L - 1, 0], kf[0, 128 + 5, 0]) / np.sqrt(d) / np.log(2.0)
+    lg2 = np.einsum("d,d->", qf[0, L - 1, 0], kf[0, 256 + 5, 0]) / np.sqrt(d) / np.log(2.0)
+    assert lg > 8.5 and lg2 - lg > 8.5
+    got = run(G, q, k, v, 1.0e6)
+    ref = R.prefill_ref(q, k, v, 1.0e6)
+    assert_close(got, ref, f"spiked prefill B={B} L={L} d={d}")
+
+
 def sample_rows(L, rng, n=24):
     fixed = {0, 1, 127, 128, 129, 255, 256, L // 2, L - 2, L - 1}
     rows = {r for r in fixed if 0 <= r < L} | set(rng.integers(0, L, n).tolist())
