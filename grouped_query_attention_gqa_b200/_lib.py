@@ -65,6 +65,9 @@ def load() -> ctypes.CDLL:
     lib.gqa_strerror.restype = ctypes.c_char_p
     lib.gqa_abi_version.argtypes = []
     lib.gqa_abi_version.restype = i
+    ip = ctypes.POINTER(ctypes.c_int)
+    lib.gqa_prefill_schedule.argtypes = [i, i, i, i, i, ip, ip, i, ip]
+    lib.gqa_prefill_schedule.restype = i
     _lib = lib
     return lib
 
@@ -273,3 +276,21 @@ def set_timing_events(start=None, stop=None) -> None:
 
 def release() -> None:
     load().gqa_release()
+
+
+def prefill_schedule(B: int, L: int, h_q: int, h_kv: int, grid: int):
+    """The attention work schedule gqa_prefill uses for this shape over `grid` CTAs (host only).
+
+    Returns (lists, snake): lists[c] is CTA c's item list in order; snake is True where the library keeps
+    its round-robin order instead (the lists are then those of the packing it compared against).
+    """
+    lib = load()
+    snake = ctypes.c_int(0)
+    n = lib.gqa_prefill_schedule(B, L, h_q, h_kv, grid, None, None, 0, ctypes.byref(snake))
+    if n < 0:
+        raise GQAError(n, "gqa_prefill_schedule")
+    g = min(grid, n)
+    starts = (ctypes.c_int * (g + 1))()
+    items = (ctypes.c_int * max(n, 1))()
+    lib.gqa_prefill_schedule(B, L, h_q, h_kv, grid, starts, items, n, ctypes.byref(snake))
+    return [list(items[starts[c]:starts[c + 1]]) for c in range(g)], bool(snake.value)

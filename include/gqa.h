@@ -213,6 +213,25 @@ GQA_API int gqa_set_stream(void* cuda_stream);
  */
 GQA_API int gqa_last_error(void);
 
+/*
+ * gqa_prefill_schedule -- how gqa_prefill and gqa_prefill_rotated deal their attention work out over `grid`
+ * persistent CTAs (one per SM: pass the SM count), computed on the host exactly as the library does it;
+ * no device is needed.  For inspection and tests.
+ * The work items are pairs of 128-row query tiles of one (batch row, KV group): item w covers the tiles
+ * 2(w / (B*h_kv)) and 2(w / (B*h_kv)) + 1 of the group b*h_kv + u = w mod (B*h_kv), whose tiles are listed
+ * by query tile descending, then head ascending (causal masking: tile index i needs L/128 - i/g key tiles).
+ * With more items than CTAs, the items are packed by best fit decreasing on (key tiles + a fixed
+ * per-item cost), each CTA taking its items in the listed order; where the plain round-robin order is
+ * within 2 % of that packing it is kept instead (*snake = 1) and the lists are those of the packing only.
+ *   starts  [min(grid, items) + 1] CTA c's items are items[starts[c] .. starts[c+1])   (caller-owned)
+ *   items   [items]                                                                   (caller-owned)
+ *   capacity  the room in items; the arrays are written only when it suffices (and both are non-null)
+ * Returns the number of items (>= 0), or GQA_ERR_DIMS for non-positive sizes, h_q % h_kv != 0 or sizes
+ * gqa_prefill rejects.
+ */
+GQA_API int gqa_prefill_schedule(int B, int L, int h_q, int h_kv, int grid, int* starts, int* items, int capacity,
+                                 int* snake);
+
 /* Frees the internal workspaces (and the cos / sin table) of every device this process used (synchronises each). */
 GQA_API void gqa_release(void);
 

@@ -1,0 +1,94 @@
+"""Host logic of the attention work schedule (gqa_prefill_schedule; no device needed).
+
+The persistent attention kernel walks per-CTA lists of work items, each a pair of 128-row query tiles of
+one (batch row, KV group).  These tests check the lists the library builds against the item enumeration
+(causal key-tile counts computed here from the shapes), not against its own code.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+
+import grouped_query_attention_gqa_b200 as G
+from grouped_query_attention_gqa_b200 import _lib
+
+
+def item_tiles(B, L, h_q, h_kv):
+    """Key tiles of every item: the group's query tiles listed by tile descending, head ascending, paired."""
+    nq = (L + 127) // 128
+    g = h_q // h_kv
+    tpg = nq * g
+    total = (tpg + 1) // 2 * B * h_kv
+    out = []
+    for w in range(total):
+        pair = w // (B * h_kv)
+        i0, i1 = 2 * pair, 2 * pair + 1
+        out.append((nq - i0 // g if i0 < tpg else 0) + (nq - i1 // g if i1 < tpg else 0))
+    return np.array(out)
+
+
+def snake_loads(tiles, grid):
+    load = np.zeros(grid, dtype=np.int64)
+    for w, t in enumerate(tiles):
+        r, c = divmod(w, grid)
+        load[grid - 1 - c if r & 1 else c] += t
+    return load
+
+
+SHAPES = [(1, 4096, 28, 4), (2, 4096, 28, 4), (1, 700, 28, 4), (1, 128, 14, 2), (3, 1000, 7, 1),
+          (1, 8192, 28, 4), (4, 4096, 64, 8), (2, 300, 8, 8)]
+
+
+@pytest.mark.parametrize("B,L,h_q,h_kv", SHAPES)
+def test_every_item_exactly_once_heaviest_first(B, L, h_q, h_kv):
+    tiles = item_tiles(B, L, h_q, h_kv)
+    lists, _ = G.prefill_schedule(B, L, h_q, h_kv, 148)
+    assert len(lists) == min(148, len(tiles))
+    flat = np.concatenate([np.array(l, dtype=np.int64) for l in lists])
+    assert np.array_equal(np.sort(flat), np.arange(len(tiles)))
+    for l in lists:
+        assert np.all(np.diff(tiles[l]) <= 0)   # each CTA takes its heaviest item first
+
+
+def test_packing_balances_the_headline_shape():
+    """Qwen2-7B at L=4096: 448 items over 148 CTAs.  Round-robin leaves the busiest CTA ~10 % above the
+    mean number of key tiles; the packing is used there and its busiest CTA carries fewer key tiles."""
+    B, L, h_q, h_kv = 1, 4096, 28, 4
+    tiles = item_tiles(B, L, h_q, h_kv)
+    lists, snake = G.prefill_schedule(B, L, h_q, h_kv, 148)
+    assert not snake
+    packed = np.array([tiles[l].sum() for l in lists])
+    rr = snake_loads(tiles, 148)
+    assert rr.max() > 1.09 * tiles.sum() / 148
+    assert packed.max() < rr.max()
+    assert packed.sum() == tiles.sum()
+
+
+@pytest.mark.parametrize("B,L,h_q,h_kv", [(1, 32768, 28, 4), (4, 8192, 64, 8), (1, 16384, 28, 4)])
+def test_round_robin_kept_where_already_balanced(B, L, h_q, h_kv):
+    tiles = item_tiles(B, L, h_q, h_kv)
+    _, snake = G.prefill_schedule(B, L, h_q, h_kv, 148)
+    assert snake
+    rr = snake_loads(tiles, 148)
+    assert rr.max() <= 1.01 * tiles.sum() / 148 + tiles.max()
+
+
+def test_fewer_items_than_ctas():
+    lists, _ = G.prefill_schedule(1, 128, 14, 2, 148)   # 8 items (2 groups x 4 pairs): one per CTA
+    assert all(len(l) == 1 for l in lists)
+
+
+@pytest.mark.parametrize("args", [(0, 16, 28, 4, 148), (1, 0, 28, 4, 148), (1, 16, 28, 5, 148), (1, 16, 28, 4, 0),
+                                  (1, 16, 0, 4, 148), (1, 16, 28, -4, 148)])
+def test_schedule_validation(args):
+    lib = _lib.load()
+    assert lib.gqa_prefill_schedule(*args, None, None, 0, None) == -2   # GQA_ERR_DIMS
+
+
+def test_small_capacity_leaves_arrays_untouched():
+    lib = _lib.load()
+    starts = (ctypes.c_int * 149)(*([-7] * 149))
+    items = (ctypes.c_int * 4)(*([-7] * 4))
+    n = lib.gqa_prefill_schedule(1, 4096, 28, 4, 148, starts, items, 4, None)
+    assert n == 448
+    assert list(starts) == [-7] * 149 and list(items) == [-7] * 4
