@@ -61,7 +61,10 @@ extern "C" {
  * Positions are 0 .. L-1 in every batch row.  d in {64, 128}; h_q % h_kv == 0; any L >= 1
  * (a ragged last tile is handled).  B == 0 or L == 0 is a no-op that returns GQA_OK.
  * Uses an internal device workspace (rotated Q and K, B*(h_q+h_kv)*L*d*2 bytes), grown on
- * demand and kept until gqa_release().
+ * demand and kept until gqa_release().  The first call for a new (B, L, h_q, h_kv) also plans
+ * the attention kernel's work schedule on the host and copies it to the device (a few KB, kept
+ * until the shape changes; see gqa_prefill_schedule): to capture calls into a CUDA graph, make
+ * one call of the shape before capturing.
  * theta is the RoPE base (Qwen2: 1e6).
  */
 GQA_API int gqa_prefill(const void* q, const void* k, const void* v, void* out,
