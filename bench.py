@@ -557,7 +557,8 @@ def run_ours(args):
     allb = decode_bytes(total_rows, wd)
     line = None
     if rank == 0:
-        achieved_t = fl / (attn_mean * 1e-3) / 1e12 if do_p else None
+        # --only decode: attn_mean is NaN, and the prefill roofline below is dropped from the line
+        achieved_t = fl / (attn_mean * 1e-3) / 1e12
         achieved_b = allb / (split_mean * 1e-3) / 1e9
         line = {
             "metric": METRIC,
@@ -581,7 +582,7 @@ def run_ours(args):
                          "frac_of_spec": achieved_t / SPEC_BF16_TFLOPS,
                          "exp_per_launch": wp.B * wp.h_q * wp.L * (wp.L + 1) // 2,
                          "exp_per_s": wp.B * wp.h_q * wp.L * (wp.L + 1) / 2 / (attn_mean * 1e-3)},
-            "cpu_baseline": cpu_baseline(wp) if (world == 1 and not args.no_cpu_baseline) else None,
+            "cpu_baseline": cpu_baseline(wp) if (world == 1 and do_p and not args.no_cpu_baseline) else None,
             "only": args.only,
             "e2e": {"value": world * fl / (e2e_pre * 1e-3) / 1e12, "unit": "TFLOP/s",
                     "h2d_bytes_per_step": sum(x.numel() * x.element_size() for x in (q, k, v)),

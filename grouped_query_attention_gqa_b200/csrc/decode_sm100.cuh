@@ -87,6 +87,8 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(const int* __restric
     __shared__ int64_t warp_tot[PLAN_THREADS / 32];
     __shared__ int64_t carry;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    // The split kernel may launch now: it waits for this grid's offsets with griddepcontrol.wait.
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     if (tid == 0) {
         carry = 0;
         off[0] = 0;
@@ -220,6 +222,10 @@ __global__ void __launch_bounds__(WARPS * 32, CTAS_PER_SM) split_kernel(const Pa
         fence_mbar_init();
     }
     __syncthreads();   // the last CTA-wide barrier: warps are independent from here on
+    // Launched as a programmatic dependent of plan_kernel: everything above overlaps it; the offsets it
+    // writes are read only after its grid has completed.  The combine kernel may launch from here on.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
     const int64_t N = p.off[p.B];
     const int64_t start = slice_start(N, w, p.P);
@@ -448,6 +454,8 @@ __global__ void __launch_bounds__(COMBINE_THREADS) combine_kernel(const Params p
     __shared__ const float* s_ptr[CHUNK];
     __shared__ float s_M[HB], s_L[HB];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    // A programmatic dependent of split_kernel: its partials are read only after its grid has completed.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const int hb = blockIdx.x % p.n_hb;
     const int u = (blockIdx.x / p.n_hb) % p.h_kv;
     const int b = blockIdx.x / (p.n_hb * p.h_kv);

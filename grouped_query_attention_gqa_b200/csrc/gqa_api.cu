@@ -516,6 +516,43 @@ int launch_proj(DeviceState* st, const void* attn, const void* w_o, const void* 
     return run_gemm<bn>(st, proj_kernel<bn>, 4u, st->proj_maps, p);
 }
 
+// The decode step's three kernels: plan (offsets), split (one partial per piece), combine (merge).
+// Split and combine are programmatic dependents of the kernel before them: their CTAs may start
+// (barrier and RoPE-table set-up) while it drains, and wait for its results with griddepcontrol.wait.
+// With timing events around the split kernel (`marks` and events set) the launches are plain.
+template <int D>
+int launch_decode_chain(const gqa::decode::Params& p, const int* seqlens, int64_t* off, int split_grid, bool marks) {
+    using namespace gqa::decode;
+    using C = Cfg<D>;
+    const long long cgrid = static_cast<long long>(p.B) * p.h_kv * p.n_hb;
+    if (cgrid > 0x7fffffffLL) return GQA_ERR_DIMS;
+    if (cudaFuncSetAttribute(split_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
+        return GQA_ERR_LAUNCH;
+    const bool timed = marks && g_ev_start && g_ev_stop;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.stream = g_stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 0;
+    cfg.gridDim = dim3(1);
+    cfg.blockDim = dim3(PLAN_THREADS);
+    if (cudaLaunchKernelEx(&cfg, plan_kernel, seqlens, off, p.B, p.err) != cudaSuccess) return GQA_ERR_LAUNCH;
+    if (marks) mark(g_ev_start);
+    cfg.numAttrs = timed ? 0 : 1;
+    cfg.gridDim = dim3(split_grid);
+    cfg.blockDim = dim3(WARPS * 32);
+    cfg.dynamicSmemBytes = C::SMEM;
+    if (cudaLaunchKernelEx(&cfg, split_kernel<D>, p) != cudaSuccess) return GQA_ERR_LAUNCH;
+    if (marks) mark(g_ev_stop);
+    cfg.gridDim = dim3(static_cast<unsigned>(cgrid));
+    cfg.blockDim = dim3(COMBINE_THREADS);
+    cfg.dynamicSmemBytes = 0;
+    if (cudaLaunchKernelEx(&cfg, combine_kernel<D>, p) != cudaSuccess) return GQA_ERR_LAUNCH;
+    return GQA_OK;
+}
+
 // Packed cache (bt == nullptr) or paged cache through the block table bt [B, max_pages].
 template <int D>
 int launch_decode(DeviceState* st, const void* q, const void* kc, const void* vc, const int* seqlens, void* out,
@@ -555,19 +592,7 @@ int launch_decode(DeviceState* st, const void* q, const void* kc, const void* vc
     p.scale_log2 *= rope_mscale() * rope_mscale();   // YaRN temperature (1 without scaling)
     p.err = st->err;
 
-    plan_kernel<<<1, PLAN_THREADS, 0, g_stream>>>(seqlens, static_cast<int64_t*>(st->dws), B, st->err);
-    if (cudaGetLastError() != cudaSuccess) return GQA_ERR_LAUNCH;
-    if (cudaFuncSetAttribute(split_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
-        return GQA_ERR_LAUNCH;
-    mark(g_ev_start);
-    split_kernel<D><<<G * groups, WARPS * 32, C::SMEM, g_stream>>>(p);
-    if (cudaGetLastError() != cudaSuccess) return GQA_ERR_LAUNCH;
-    mark(g_ev_stop);
-    const long long cgrid = static_cast<long long>(B) * groups;
-    if (cgrid > 0x7fffffffLL) return GQA_ERR_DIMS;
-    combine_kernel<D><<<static_cast<unsigned>(cgrid), COMBINE_THREADS, 0, g_stream>>>(p);
-    if (cudaGetLastError() != cudaSuccess) return GQA_ERR_LAUNCH;
-    return GQA_OK;
+    return launch_decode_chain<D>(p, seqlens, static_cast<int64_t*>(st->dws), G * groups, true);
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -633,17 +658,7 @@ int launch_decode_fixed_scratch(DeviceState* st, const void* q, const void* kc, 
     p.scale_log2 *= rope_mscale() * rope_mscale();   // YaRN temperature (1 without scaling)
     p.err = st->err;
 
-    plan_kernel<<<1, PLAN_THREADS, 0, g_stream>>>(seqlens, static_cast<int64_t*>(st->fixed_scratch), B, st->err);
-    if (cudaGetLastError() != cudaSuccess) return GQA_ERR_LAUNCH;
-    if (cudaFuncSetAttribute(split_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
-        return GQA_ERR_LAUNCH;
-    split_kernel<D><<<G * groups, WARPS * 32, C::SMEM, g_stream>>>(p);
-    if (cudaGetLastError() != cudaSuccess) return GQA_ERR_LAUNCH;
-    const long long cgrid = static_cast<long long>(B) * groups;
-    if (cgrid > 0x7fffffffLL) return GQA_ERR_DIMS;
-    combine_kernel<D><<<static_cast<unsigned>(cgrid), COMBINE_THREADS, 0, g_stream>>>(p);
-    if (cudaGetLastError() != cudaSuccess) return GQA_ERR_LAUNCH;
-    return GQA_OK;
+    return launch_decode_chain<D>(p, seqlens, static_cast<int64_t*>(st->fixed_scratch), G * groups, false);
 }
 
 }  // namespace
