@@ -70,21 +70,6 @@ constexpr float kRescaleThreshold = 8.0f;   // log2 units: O is rescaled only wh
 #ifndef GQA_EXP_POLY_OF_8
 #define GQA_EXP_POLY_OF_8 1
 #endif
-// 1: round P to bf16 with integer ops instead of the conversion instruction.
-#ifndef GQA_PACK_INT
-#define GQA_PACK_INT 0
-#endif
-// 1: P is truncated to bf16 (one byte permute per pair, off the conversion unit) and the row sum l
-// accumulates the same truncated values, so the normalisation matches the weights the MMA uses.
-#ifndef GQA_PACK_TRUNC
-#define GQA_PACK_TRUNC 0
-#endif
-// Epilogue: each softmax warp stages its 32 output rows, one 64-column half at a time, in a 4 KB
-// slot of its own and writes them with TMA stores, so the Q' tile is handed back to the producer as
-// soon as the pair's last S has finished (GQA_EPILOGUE_TMA 1).  0: every thread stores its row directly.
-#ifndef GQA_EPILOGUE_TMA
-#define GQA_EPILOGUE_TMA 1
-#endif
 #ifndef GQA_PREP_POS
 #define GQA_PREP_POS 8
 #endif
@@ -229,14 +214,6 @@ __global__ void __launch_bounds__(PREP_THREADS, GQA_PREP_MIN_CTAS) prep_kernel(c
     }
 }
 
-__device__ __forceinline__ uint32_t pack_p(float lo, float hi) {
-#if GQA_PACK_INT
-    return pack_bf16x2_int(lo, hi);
-#else
-    return pack_bf16x2(lo, hi);
-#endif
-}
-
 // P = 2^(s * scale_log2 - m) for one row of 128 scores, stored as bf16 pairs into the first 64
 // columns of the S region (chunk c overwrites S columns 16c.., already in registers); returns the
 // row sum of the fp32 values.  POLY: part of the exponentials on the FMA pipe (never on a tile
@@ -261,7 +238,7 @@ __device__ __forceinline__ float row_exp_store(const uint32_t (&sr)[4][32], floa
                 p1 = ex2(x1);
             }
             acc[(e >> 1) & 1] = f2_add(acc[(e >> 1) & 1], f2_pack(p0, p1));
-            pk[e >> 1] = pack_p(p0, p1);
+            pk[e >> 1] = pack_bf16x2(p0, p1);
         }
         tmem_st16(t_s + 16 * c, pk);
     }
@@ -445,7 +422,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             if (!ok) break;
             tc_fence_after();
             const float inv_l = 1.0f / l_run;
-#if GQA_EPILOGUE_TMA
             // Rows 32*(warp&3) .. +31 of the tile, one 64-column half per pass: stage in this warp's slot
             // (same 128-byte-swizzled layout as the output tensor map's 64 x 32 box), TMA-store, and wait
             // for the store to have read the slot before the next pass.  Rows >= L are clipped.
@@ -478,27 +454,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 __syncwarp();
             }
             tc_fence_before();
-#else
-            const int row = qtk * BM + r;
-            uint4* dst = reinterpret_cast<uint4*>(
-                p.out + ((static_cast<int64_t>(pw.b) * p.L + row) * p.h_q + headk) * D);
-#pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
-                uint32_t o[32];
-                tmem_ld32(t_o + 32 * c, o);
-                tmem_wait_ld();
-                uint32_t wv[16];
-#pragma unroll
-                for (int e = 0; e < 16; ++e)
-                    wv[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv_l, __uint_as_float(o[2 * e + 1]) * inv_l);
-                if (row < p.L) {
-#pragma unroll
-                    for (int v4 = 0; v4 < 4; ++v4)
-                        dst[4 * c + v4] = make_uint4(wv[4 * v4], wv[4 * v4 + 1], wv[4 * v4 + 2], wv[4 * v4 + 3]);
-                }
-            }
-            tc_fence_before();
-#endif
         }
     } else if (warp == WARP_TMA) {
         // ================================================================ TMA producer
