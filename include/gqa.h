@@ -17,7 +17,10 @@
  *     and the first call on a device (one-time device query).
  *   - Return value: 0 on success, or one of the negative GQA_ERR_* codes.  A failing call
  *     launches nothing and leaves `out` untouched.  Library code never traps or aborts.
- *   - Not thread-safe: the stream and the workspace are process-global state.
+ *   - Not thread-safe: the stream and the workspace are process-global state.  Calls that can
+ *     overlap on the GPU (enqueued on different streams without synchronisation between them)
+ *     share that workspace and the cached attention schedule and race: keep such calls on one
+ *     stream, or synchronise between them.
  */
 #ifndef GQA_H_
 #define GQA_H_
