@@ -339,6 +339,74 @@ def ev():
     return e
 
 
+def build_line(*, world, K, W, only, do_p, do_d, wp, wd, value_tflops, pre_mean, attn_mean, dec_mean, split_mean,
+               total_rows, page, peaks, peak_src, cpu_base, e2e_pre, e2e_dec, pre_io, dec_io, qkv_line, clocks,
+               t_wall):
+    """The JSON line of the `ours` arm from the measured numbers (no device work, so the CPU tests cover it).
+    Times in ms; pre_io / dec_io = (host->device, device->host) bytes of one end-to-end prefill / decode
+    step; a leg that did not run carries NaN, which clean() turns into null."""
+    fl = prefill_flops(wp)
+    kvb = decode_kv_bytes(total_rows, wd)
+    allb = decode_bytes(total_rows, wd)
+    # --only decode: attn_mean is NaN, and the prefill roofline below is dropped from the line
+    achieved_t = fl / (attn_mean * 1e-3) / 1e12
+    achieved_b = allb / (split_mean * 1e-3) / 1e9
+    line = {
+        "metric": METRIC,
+        "value": value_tflops,
+        "unit": "TFLOP/s",
+        "n_gpus": world, "steps": K, "warmup": W,
+        "ms_per_step": pre_mean,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic: seeded N(0,1) bf16 Q/K/V and caches drawn on the device; decode lengths U[1,32768]",
+        "config": dict(bench_config(wp, wd),
+                       timing=f"{K} headline steps without per-kernel events, interleaved with {K} steps "
+                              "with CUDA events around the attention / split kernels for the roofline"),
+        "roofline": {"kernel": "attn_kernel (prefill)", "bound": "tensor", "achieved": achieved_t,
+                     "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved_t / peaks["bf16_tflops"],
+                     "peak_source": f"{peak_src} bf16 dense (burst)",
+                     "traffic": profile_traffic("attn_kernel", wp.name),
+                     "algorithmic_flops_per_launch": fl, "ms_per_launch": attn_mean,
+                     # beside the burst peak: the sustained cuBLAS figure and the 2.25 PFLOP/s data-sheet
+                     # number, and the exponentials per launch (one per unmasked score)
+                     "frac_of_sustained": achieved_t / peaks["bf16_tflops_sustained"],
+                     "frac_of_spec": achieved_t / SPEC_BF16_TFLOPS,
+                     "exp_per_launch": wp.B * wp.h_q * wp.L * (wp.L + 1) // 2,
+                     "exp_per_s": wp.B * wp.h_q * wp.L * (wp.L + 1) / 2 / (attn_mean * 1e-3)},
+        "cpu_baseline": cpu_base,
+        "only": only,
+        "e2e": {"value": world * fl / (e2e_pre * 1e-3) / 1e12, "unit": "TFLOP/s",
+                "h2d_bytes_per_step": pre_io[0], "d2h_bytes_per_step": pre_io[1]},
+        "gpu_launches": (2 * do_p + 3 * do_d) * 2 * K + (6 * K if qkv_line else 0),
+        "qkv": qkv_line,
+        "clocks": clocks,
+        "decode": {
+            "workload": wd.desc, "total_cache_rows": total_rows,
+            "layout": f"paged: {page} rows per page, pages scattered in a seeded random order" if page
+                      else "packed",
+            "value": world * allb / (dec_mean * 1e-3) / 1e9, "unit": "GB/s",
+            "kv_gbs": world * kvb / (dec_mean * 1e-3) / 1e9,
+            "ms_per_step": dec_mean,
+            "roofline": {"kernel": "split_kernel (decode)", "bound": "hbm", "achieved": achieved_b,
+                         "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": achieved_b / peaks["hbm_gbs"],
+                         "peak_source": f"{peak_src} HBM copy",
+                         "traffic": profile_traffic("split_kernel", DECODE_WORKLOAD + (f"-paged{page}" if page else "")),
+                         "algorithmic_bytes_per_launch": allb, "ms_per_launch": split_mean},
+            "e2e": {"value": world * allb / (e2e_dec * 1e-3) / 1e9, "unit": "GB/s",
+                    "h2d_bytes_per_step": dec_io[0], "d2h_bytes_per_step": dec_io[1],
+                    "note": "the KV cache is resident device state; the step's inputs are q, the lengths"
+                            + (" and the block table" if page else "")},
+        },
+        "wall_s_timed_region": t_wall,
+        "impl": "ours",
+    }
+    if not do_p:   # --only decode: the line carries the decode half alone
+        line["roofline"] = line["e2e"] = line["cpu_baseline"] = None
+    if not do_d:   # --only prefill
+        line["decode"] = None
+    return line
+
+
 def run_ours(args):
     rank, local, world = dist_env()
     dist_init(world)
@@ -553,68 +621,17 @@ def run_ours(args):
         del xq, wqkv, bqkv, qo, w_o, x_in, y_out
 
     peaks, peak_src = load_peaks()
-    kvb = decode_kv_bytes(total_rows, wd)
-    allb = decode_bytes(total_rows, wd)
     line = None
     if rank == 0:
-        # --only decode: attn_mean is NaN, and the prefill roofline below is dropped from the line
-        achieved_t = fl / (attn_mean * 1e-3) / 1e12
-        achieved_b = allb / (split_mean * 1e-3) / 1e9
-        line = {
-            "metric": METRIC,
-            "value": value_tflops,
-            "unit": "TFLOP/s",
-            "n_gpus": world, "steps": K, "warmup": W,
-            "ms_per_step": pre_mean,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-            "data": "synthetic: seeded N(0,1) bf16 Q/K/V and caches drawn on the device; decode lengths U[1,32768]",
-            "config": dict(bench_config(wp, wd),
-                           timing=f"{K} headline steps without per-kernel events, interleaved with {K} steps "
-                                  "with CUDA events around the attention / split kernels for the roofline"),
-            "roofline": {"kernel": "attn_kernel (prefill)", "bound": "tensor", "achieved": achieved_t,
-                         "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved_t / peaks["bf16_tflops"],
-                         "peak_source": f"{peak_src} bf16 dense (burst)",
-                         "traffic": profile_traffic("attn_kernel", wp.name),
-                         "algorithmic_flops_per_launch": fl, "ms_per_launch": attn_mean,
-                         # beside the burst peak: the sustained cuBLAS figure and the 2.25 PFLOP/s data-sheet
-                         # number, and the exponentials per launch (one per unmasked score)
-                         "frac_of_sustained": achieved_t / peaks["bf16_tflops_sustained"],
-                         "frac_of_spec": achieved_t / SPEC_BF16_TFLOPS,
-                         "exp_per_launch": wp.B * wp.h_q * wp.L * (wp.L + 1) // 2,
-                         "exp_per_s": wp.B * wp.h_q * wp.L * (wp.L + 1) / 2 / (attn_mean * 1e-3)},
-            "cpu_baseline": cpu_baseline(wp) if (world == 1 and do_p and not args.no_cpu_baseline) else None,
-            "only": args.only,
-            "e2e": {"value": world * fl / (e2e_pre * 1e-3) / 1e12, "unit": "TFLOP/s",
-                    "h2d_bytes_per_step": sum(x.numel() * x.element_size() for x in (q, k, v)),
-                    "d2h_bytes_per_step": out.numel() * out.element_size()},
-            "gpu_launches": (2 * do_p + 3 * do_d) * 2 * K + (6 * K if qkv_line else 0),
-            "qkv": qkv_line,
-            "clocks": sampler.summary(),
-            "decode": {
-                "workload": wd.desc, "total_cache_rows": total_rows,
-                "layout": f"paged: {page} rows per page, pages scattered in a seeded random order" if page
-                          else "packed",
-                "value": world * allb / (dec_mean * 1e-3) / 1e9, "unit": "GB/s",
-                "kv_gbs": world * kvb / (dec_mean * 1e-3) / 1e9,
-                "ms_per_step": dec_mean,
-                "roofline": {"kernel": "split_kernel (decode)", "bound": "hbm", "achieved": achieved_b,
-                             "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": achieved_b / peaks["hbm_gbs"],
-                             "peak_source": f"{peak_src} HBM copy",
-                             "traffic": profile_traffic("split_kernel", DECODE_WORKLOAD + (f"-paged{page}" if page else "")),
-                             "algorithmic_bytes_per_launch": allb, "ms_per_launch": split_mean},
-                "e2e": {"value": world * allb / (e2e_dec * 1e-3) / 1e9, "unit": "GB/s",
-                        "h2d_bytes_per_step": qd.numel() * 2 + s.numel() * 4 + (table.numel() * 4 if page else 0),
-                        "d2h_bytes_per_step": outd.numel() * 2,
-                        "note": "the KV cache is resident device state; the step's inputs are q, the lengths"
-                                + (" and the block table" if page else "")},
-            },
-            "wall_s_timed_region": t_wall,
-            "impl": "ours",
-        }
-        if not do_p:   # --only decode: the line carries the decode half alone
-            line["roofline"] = line["e2e"] = line["cpu_baseline"] = None
-        if not do_d:   # --only prefill
-            line["decode"] = None
+        line = build_line(
+            world=world, K=K, W=W, only=args.only, do_p=do_p, do_d=do_d, wp=wp, wd=wd, value_tflops=value_tflops,
+            pre_mean=pre_mean, attn_mean=attn_mean, dec_mean=dec_mean, split_mean=split_mean, total_rows=total_rows,
+            page=page, peaks=peaks, peak_src=peak_src,
+            cpu_base=cpu_baseline(wp) if (world == 1 and do_p and not args.no_cpu_baseline) else None,
+            e2e_pre=e2e_pre, e2e_dec=e2e_dec,
+            pre_io=(sum(x.numel() * x.element_size() for x in (q, k, v)), out.numel() * out.element_size()),
+            dec_io=(qd.numel() * 2 + s.numel() * 4 + (table.numel() * 4 if page else 0), outd.numel() * 2),
+            qkv_line=qkv_line, clocks=sampler.summary(), t_wall=t_wall)
     if torch.distributed.is_initialized():
         barrier()
         torch.distributed.destroy_process_group()
