@@ -61,10 +61,10 @@ struct DeviceState {
     unsigned gemm_ready = 0;   // bit per GEMM kernel instantiation whose shared-memory size is set
     const void* qkv_key[2] = {nullptr, nullptr};
     long long qkv_dims[4] = {0, 0, 0, 0};
-    CUtensorMap qkv_maps[2];
+    CUtensorMap qkv_maps[3];
     const void* proj_key[2] = {nullptr, nullptr};
     long long proj_dims[4] = {0, 0, 0, 0};
-    CUtensorMap proj_maps[2];
+    CUtensorMap proj_maps[3];
 };
 
 DeviceState g_dev[kMaxDevices];
@@ -422,7 +422,8 @@ int ensure_rope_table(DeviceState* st, int L, float theta) {
     return GQA_OK;
 }
 
-// X [T, K] and W [N, K] tensor maps of a projection GEMM with tile width bn, reused while the key matches.
+// X [T, K] and W [N, K] tensor maps of a projection GEMM with tile width bn, and W again with the box of
+// a tail unit (TAIL_BN rows); reused while the key matches.
 bool gemm_maps(CUtensorMap* maps, const void** key, long long* dims, const void* x, const void* w, long long T,
                int K, long long N, int bn) {
     using namespace gqa::qkv;
@@ -436,6 +437,8 @@ bool gemm_maps(CUtensorMap* maps, const void** key, long long* dims, const void*
     const cuuint64_t dw[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(N)};
     const cuuint32_t bw[2] = {BK, static_cast<cuuint32_t>(bn)};
     if (!encode_bf16(&maps[1], const_cast<void*>(w), 2, dw, sx, bw)) return false;
+    const cuuint32_t bt[2] = {BK, static_cast<cuuint32_t>(TAIL_BN)};
+    if (!encode_bf16(&maps[2], const_cast<void*>(w), 2, dw, sx, bt)) return false;
     key[0] = x;
     key[1] = w;
     dims[0] = T;
@@ -446,9 +449,12 @@ bool gemm_maps(CUtensorMap* maps, const void** key, long long* dims, const void*
 }
 
 // Launch one instantiation of the persistent GEMM (the kernel `fn`, tile width BN) over p.n_tiles tiles.
+// With `split_tail`, a last wave at most a quarter full is split into BN / TAIL_BN-column units, so that
+// it occupies four times as many CTAs for a quarter of the time each (the output projection: the
+// 4096 x 3584 product is 448 tiles = 3 waves of 148 and 4 tiles).
 template <int BN>
-int run_gemm(DeviceState* st, void (*fn)(CUtensorMap, CUtensorMap, gqa::qkv::Params), unsigned ready_bit,
-             const CUtensorMap* maps, const gqa::qkv::Params& p) {
+int run_gemm(DeviceState* st, void (*fn)(CUtensorMap, CUtensorMap, CUtensorMap, gqa::qkv::Params),
+             unsigned ready_bit, const CUtensorMap* maps, gqa::qkv::Params p, bool split_tail) {
     using namespace gqa::qkv;
     if (!(st->gemm_ready & ready_bit)) {
         if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, Tile<BN>::DYN) != cudaSuccess)
@@ -456,8 +462,17 @@ int run_gemm(DeviceState* st, void (*fn)(CUtensorMap, CUtensorMap, gqa::qkv::Par
         st->gemm_ready |= ready_bit;
     }
     const int grid = p.n_tiles < st->num_sms ? p.n_tiles : st->num_sms;
+    const int last = p.n_tiles % grid;   // tiles in a partly filled last wave
+    constexpr int SPLIT = BN / TAIL_BN;
+    p.n_main = p.n_tiles;
+    p.tail_split = 1;
+    if (split_tail && SPLIT > 1 && last > 0 && last * SPLIT <= grid) {
+        p.n_main = p.n_tiles - last;
+        p.tail_split = SPLIT;
+    }
+    p.n_units = p.n_main + (p.n_tiles - p.n_main) * p.tail_split;
     mark(g_ev_start);
-    fn<<<grid, NUM_THREADS, Tile<BN>::DYN, g_stream>>>(maps[0], maps[1], p);
+    fn<<<grid, NUM_THREADS, Tile<BN>::DYN, g_stream>>>(maps[0], maps[1], maps[2], p);
     if (cudaGetLastError() != cudaSuccess) return GQA_ERR_LAUNCH;
     mark(g_ev_stop);
     return GQA_OK;
@@ -491,7 +506,7 @@ int launch_qkv(DeviceState* st, const void* x, const void* w, const void* bias, 
     p.n_tiles = static_cast<int>(mtiles * p.n_ntiles);
     p.kblocks = (d_model + BK - 1) / BK;
     p.err = st->err;
-    return run_gemm<bn>(st, qkv_kernel<D, bn>, D == 128 ? 1u : 2u, st->qkv_maps, p);
+    return run_gemm<bn>(st, qkv_kernel<D, bn>, D == 128 ? 1u : 2u, st->qkv_maps, p, false);
 }
 
 // Output projection + residual: out [T, d_model] = attn [T, d_in] w_o [d_model, d_in]^T (+ resid).
@@ -513,7 +528,7 @@ int launch_proj(DeviceState* st, const void* attn, const void* w_o, const void* 
     p.n_tiles = static_cast<int>(mtiles * p.n_ntiles);
     p.kblocks = (d_in + BK - 1) / BK;
     p.err = st->err;
-    return run_gemm<bn>(st, proj_kernel<bn>, 4u, st->proj_maps, p);
+    return run_gemm<bn>(st, proj_kernel<bn>, 4u, st->proj_maps, p, true);
 }
 
 // The decode step's three kernels: plan (offsets), split (one partial per piece), combine (merge).

@@ -67,8 +67,35 @@ struct Params {
     __nv_bfloat16* out;          // output projection: out [T, N] (may be resid itself)
     int T, L, N, h_q, h_kv;
     int n_ntiles, n_tiles, kblocks;
+    // Work units: tiles 0 .. n_main-1 whole (BN columns); each later tile split into tail_split units of
+    // BN / tail_split columns, so that a last wave with few tiles is spread over more CTAs.  n_units in all.
+    int n_main, tail_split, n_units;
     int* err;
 };
+
+// Columns of a tail unit (MMA N); its weight rows come through a tensor map whose box is this high.
+constexpr int TAIL_BN = 64;
+
+// Rows [mt * BM, +BM) and columns [n0, n0 + width) of work unit u.
+struct Unit {
+    int mt, n0, width;
+};
+template <int BN, bool TAIL>
+__device__ __forceinline__ Unit unit_of(const Params& p, int u) {
+    Unit r;
+    if (!TAIL || u < p.n_main) {
+        r.mt = u / p.n_ntiles;
+        r.n0 = (u % p.n_ntiles) * BN;
+        r.width = BN;
+    } else {
+        const int v = u - p.n_main;
+        const int tile = p.n_main + v / p.tail_split;
+        r.mt = tile / p.n_ntiles;
+        r.width = BN / p.tail_split;
+        r.n0 = (tile % p.n_ntiles) * BN + (v % p.tail_split) * r.width;
+    }
+    return r;
+}
 
 struct alignas(8) Shared {
     uint64_t full[MAX_STAGES], empty[MAX_STAGES];
@@ -188,16 +215,17 @@ __device__ __forceinline__ void store_head(const Params& p, float (&y)[D], int n
     }
 }
 
-// The output projection's epilogue: 128 columns of one row per lane, + the residual, stored as rows.
+// The output projection's epilogue: W columns of one row per lane, + the residual, stored as rows.
 // The residual is read directly, each thread its own row: measured faster than reading whole rows
 // through the staging buffer, whose round trip sits on the epilogue's critical path.
-__device__ __forceinline__ void store_resid(const Params& p, float (&y)[128], int n0, int t, bool valid,
+template <int W>
+__device__ __forceinline__ void store_resid(const Params& p, float (&y)[W], int n0, int t, bool valid,
                                             uint8_t* stage, int lane) {
     const int64_t at = static_cast<int64_t>(t) * p.N + n0;
     if (p.resid && valid) {
         const uint4* rr = reinterpret_cast<const uint4*>(p.resid + at);
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
+        for (int c = 0; c < W / 8; ++c) {
             const uint4 w = rr[c];
             const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
@@ -207,7 +235,7 @@ __device__ __forceinline__ void store_resid(const Params& p, float (&y)[128], in
             }
         }
     }
-    store_rows<128>(stage, valid ? p.out + at : nullptr, y, lane);
+    store_rows<W>(stage, valid ? p.out + at : nullptr, y, lane);
 }
 
 enum Epilogue { kQKV = 0, kResidual = 1 };
@@ -216,7 +244,8 @@ enum Epilogue { kQKV = 0, kResidual = 1 };
 // The persistent GEMM: Y[T, N] = X[T, K] W[N, K]^T with the epilogue EPI.  For kQKV, D is the head size
 // (tiles are processed head by head); for kResidual, D = 128 (tiles are processed 128 columns at a time).
 template <int D, int EPI, int BN_>
-__device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtensorMap& tm_w, const Params& p) {
+__device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtensorMap& tm_w, const CUtensorMap& tm_wt,
+                                          const Params& p) {
     constexpr int BN = Tile<BN_>::BN;
     constexpr int STAGES = Tile<BN_>::STAGES;
     constexpr int STAGE_BYTES = Tile<BN_>::STAGE_BYTES;
@@ -246,6 +275,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtenso
     if (warp == WARP_TMA && lane == 0) {
         prefetch_tensormap(&tm_x);
         prefetch_tensormap(&tm_w);
+        if (p.tail_split > 1) prefetch_tensormap(&tm_wt);
     }
     tc_fence_before();
     __syncthreads();
@@ -258,18 +288,19 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtenso
         if (lane == 0) {
             uint32_t it = 0;   // K blocks issued (ring position)
             bool ok = true;
-            for (int tile = blockIdx.x; ok && tile < p.n_tiles; tile += gridDim.x) {
-                const int mt = tile / p.n_ntiles, nt = tile % p.n_ntiles;
+            for (int u = blockIdx.x; ok && u < p.n_units; u += gridDim.x) {
+                const Unit un = unit_of<BN, EPI == kResidual>(p, u);
+                const bool whole = un.width == BN;
                 for (int kb = 0; kb < p.kblocks; ++kb) {
                     const int s = static_cast<int>(it % STAGES);
                     if (it >= STAGES && !mbar_wait(&sh.empty[s], ((it / STAGES) - 1) & 1, p.err, abort)) {
                         ok = false;
                         break;
                     }
-                    mbar_arrive_expect_tx(&sh.full[s], STAGE_BYTES);
+                    mbar_arrive_expect_tx(&sh.full[s], whole ? STAGE_BYTES : A_BYTES + TAIL_BN * BK * 2);
                     uint8_t* a = smem + s * STAGE_BYTES;
-                    tma_load_2d(a, &tm_x, &sh.full[s], kb * BK, mt * BM);
-                    tma_load_2d(a + A_BYTES, &tm_w, &sh.full[s], kb * BK, nt * BN);
+                    tma_load_2d(a, &tm_x, &sh.full[s], kb * BK, un.mt * BM);
+                    tma_load_2d(a + A_BYTES, whole ? &tm_w : &tm_wt, &sh.full[s], kb * BK, un.n0);
                     ++it;
                 }
             }
@@ -280,12 +311,14 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtenso
     } else if (warp == WARP_MMA) {
         // ================================================================ MMA issuer
         if (lane == 0) {
-            constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN, false);
+            constexpr uint32_t IDESC_WHOLE = idesc_bf16_f32(BM, BN, false);
+            constexpr uint32_t IDESC_TAIL = idesc_bf16_f32(BM, TAIL_BN, false);
             const uint32_t base = smem_u32(smem);
             uint32_t it = 0;
             int local = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; ok && tile < p.n_tiles; tile += gridDim.x, ++local) {
+            for (int u = blockIdx.x; ok && u < p.n_units; u += gridDim.x, ++local) {
+                const uint32_t IDESC = unit_of<BN, EPI == kResidual>(p, u).width == BN ? IDESC_WHOLE : IDESC_TAIL;
                 const int buf = local & 1;
                 // The epilogue must have read this accumulator out (two tiles ago) before it is overwritten.
                 if (local >= 2 && !mbar_wait(&sh.acc_empty[buf], ((local >> 1) - 1) & 1, p.err, abort)) {
@@ -323,26 +356,39 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtenso
         const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
         uint8_t* stage = smem + STAGES * STAGE_BYTES + (warp - 2) * STAGING;
         int local = 0;
-        for (int tile = blockIdx.x; tile < p.n_tiles; tile += gridDim.x, ++local) {
+        for (int u = blockIdx.x; u < p.n_units; u += gridDim.x, ++local) {
             const int buf = local & 1;
             if (!__all_sync(0xffffffffu, mbar_wait(&sh.acc_full[buf], (local >> 1) & 1, p.err, abort))) break;
             tc_fence_after();
-            const int mt = tile / p.n_ntiles, nt = tile % p.n_ntiles;
-            const int t = mt * BM + r;
+            const Unit un = unit_of<BN, EPI == kResidual>(p, u);
+            const int t = un.mt * BM + r;
             const bool valid = t < p.T;
             const int b = valid ? t / p.L : 0, pos = valid ? t % p.L : 0;
-#pragma unroll 1
-            for (int hh = 0; hh < BN / D; ++hh) {
-                const int n0 = nt * BN + hh * D;
-                if (n0 >= p.N) break;
-                float acc[D];
+            if (EPI == kResidual && un.width == TAIL_BN) {
+                // A tail unit (output projection only): its 64 columns in one pass.
+                if (un.n0 < p.N) {
+                    float acc[TAIL_BN];
 #pragma unroll
-                for (int c = 0; c < D / 32; ++c)
-                    tmem_ld32(tmem + lane_base + static_cast<uint32_t>(buf * BN + hh * D + 32 * c),
-                              *reinterpret_cast<uint32_t(*)[32]>(acc + 32 * c));
-                tmem_wait_ld();
-                if (EPI == kQKV) store_head<D>(p, acc, n0, b, pos, valid, stage, lane);
-                else store_resid(p, *reinterpret_cast<float(*)[128]>(acc), n0, t, valid, stage, lane);
+                    for (int c = 0; c < TAIL_BN / 32; ++c)
+                        tmem_ld32(tmem + lane_base + static_cast<uint32_t>(buf * BN + 32 * c),
+                                  *reinterpret_cast<uint32_t(*)[32]>(acc + 32 * c));
+                    tmem_wait_ld();
+                    store_resid<TAIL_BN>(p, acc, un.n0, t, valid, stage, lane);
+                }
+            } else {
+#pragma unroll 1
+                for (int hh = 0; hh < BN / D; ++hh) {
+                    const int n0 = un.n0 + hh * D;
+                    if (n0 >= p.N) break;
+                    float acc[D];
+#pragma unroll
+                    for (int c = 0; c < D / 32; ++c)
+                        tmem_ld32(tmem + lane_base + static_cast<uint32_t>(buf * BN + hh * D + 32 * c),
+                                  *reinterpret_cast<uint32_t(*)[32]>(acc + 32 * c));
+                    tmem_wait_ld();
+                    if (EPI == kQKV) store_head<D>(p, acc, n0, b, pos, valid, stage, lane);
+                    else store_resid<128>(p, *reinterpret_cast<float(*)[128]>(acc), n0, t, valid, stage, lane);
+                }
             }
             // This thread's reads of the accumulator are complete: release it to the MMA warp.
             tc_fence_before();
@@ -360,16 +406,18 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtenso
 
 template <int D, int BN>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
-    qkv_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w, const Params p) {
-    gemm_body<D, kQKV, BN>(tm_x, tm_w, p);
+    qkv_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
+               const __grid_constant__ CUtensorMap tm_wt, const Params p) {
+    gemm_body<D, kQKV, BN>(tm_x, tm_w, tm_wt, p);
 }
 
 // Output projection + residual (page "Qwen2 architecture introduction", §4.1.3 steps 5-6):
 // out = attn W_O + X_in, with attn the concatenated heads [T, h_q d] and W_O^T [d_model, h_q d].
 template <int BN>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
-    proj_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w, const Params p) {
-    gemm_body<128, kResidual, BN>(tm_x, tm_w, p);
+    proj_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
+                const __grid_constant__ CUtensorMap tm_wt, const Params p) {
+    gemm_body<128, kResidual, BN>(tm_x, tm_w, tm_wt, p);
 }
 
 }  // namespace qkv
