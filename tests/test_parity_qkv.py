@@ -127,6 +127,11 @@ def test_qkv_then_attention_matches_gqa_prefill_on_the_raw_projection(G):
     (64, 72, 128, False, False),     # d_in not a multiple of the 64-wide K block, no residual
     (4736, 512, 1024, True, False),  # 37 x 4 tiles: exactly one full wave of 148 CTAs
     (1280, 512, 4096, True, True),   # 160 tiles: one whole wave and 12 more, in place
+    # The last wave's 12 tiles split into 64-column units, with an odd number (9) of K blocks per unit
+    (1280, 576, 4096, True, False),
+    # 150 tiles, the last two split; the last tile is half past d_model (two of its units store nothing);
+    # a ragged K block (200 = 3 x 64 + 8)
+    (1280, 200, 3712, True, True),
 ])
 def test_out_proj_small_full_output(G, T, d_in, dm, resid, inplace):
     rng = torch.Generator().manual_seed(T + d_in + dm)
