@@ -74,7 +74,11 @@ struct Params {
 };
 
 // Columns of a tail unit (MMA N); its weight rows come through a tensor map whose box is this high.
+// A tail unit's K block (A + its weight rows) fills a fraction of a ring stage, so each stage carries
+// several consecutive K blocks of it, back to back: the unit keeps as many bytes in flight as a whole
+// tile (its loads, not its MMAs, bound it).
 constexpr int TAIL_BN = 64;
+constexpr int TAIL_KB_BYTES = A_BYTES + TAIL_BN * BK * 2;   // 24 KB
 
 // Rows [mt * BM, +BM) and columns [n0, n0 + width) of work unit u.
 struct Unit {
@@ -250,6 +254,8 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtenso
     constexpr int STAGES = Tile<BN_>::STAGES;
     constexpr int STAGE_BYTES = Tile<BN_>::STAGE_BYTES;
     constexpr int TMEM_COLS = Tile<BN_>::TMEM_COLS;
+    constexpr int TAIL_PER_STAGE = STAGE_BYTES / TAIL_KB_BYTES;   // K blocks of a tail unit per stage
+    static_assert(TAIL_PER_STAGE >= 1, "a tail K block fits a stage");
     extern __shared__ uint8_t dyn_smem_raw[];
     __shared__ Shared sh;
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dyn_smem_raw) + 1023) & ~uintptr_t(1023));
@@ -290,18 +296,35 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtenso
             bool ok = true;
             for (int u = blockIdx.x; ok && u < p.n_units; u += gridDim.x) {
                 const Unit un = unit_of<BN, EPI == kResidual>(p, u);
-                const bool whole = un.width == BN;
-                for (int kb = 0; kb < p.kblocks; ++kb) {
-                    const int s = static_cast<int>(it % STAGES);
-                    if (it >= STAGES && !mbar_wait(&sh.empty[s], ((it / STAGES) - 1) & 1, p.err, abort)) {
-                        ok = false;
-                        break;
+                if (un.width == BN) {
+                    for (int kb = 0; kb < p.kblocks; ++kb) {
+                        const int s = static_cast<int>(it % STAGES);
+                        if (it >= STAGES && !mbar_wait(&sh.empty[s], ((it / STAGES) - 1) & 1, p.err, abort)) {
+                            ok = false;
+                            break;
+                        }
+                        mbar_arrive_expect_tx(&sh.full[s], STAGE_BYTES);
+                        uint8_t* a = smem + s * STAGE_BYTES;
+                        tma_load_2d(a, &tm_x, &sh.full[s], kb * BK, un.mt * BM);
+                        tma_load_2d(a + A_BYTES, &tm_w, &sh.full[s], kb * BK, un.n0);
+                        ++it;
                     }
-                    mbar_arrive_expect_tx(&sh.full[s], whole ? STAGE_BYTES : A_BYTES + TAIL_BN * BK * 2);
-                    uint8_t* a = smem + s * STAGE_BYTES;
-                    tma_load_2d(a, &tm_x, &sh.full[s], kb * BK, un.mt * BM);
-                    tma_load_2d(a + A_BYTES, whole ? &tm_w : &tm_wt, &sh.full[s], kb * BK, un.n0);
-                    ++it;
+                } else {
+                    for (int kb = 0; kb < p.kblocks; kb += TAIL_PER_STAGE) {
+                        const int s = static_cast<int>(it % STAGES);
+                        if (it >= STAGES && !mbar_wait(&sh.empty[s], ((it / STAGES) - 1) & 1, p.err, abort)) {
+                            ok = false;
+                            break;
+                        }
+                        const int nk = kb + TAIL_PER_STAGE <= p.kblocks ? TAIL_PER_STAGE : p.kblocks - kb;
+                        mbar_arrive_expect_tx(&sh.full[s], static_cast<uint32_t>(nk * TAIL_KB_BYTES));
+                        for (int q = 0; q < nk; ++q) {
+                            uint8_t* a = smem + s * STAGE_BYTES + q * TAIL_KB_BYTES;
+                            tma_load_2d(a, &tm_x, &sh.full[s], (kb + q) * BK, un.mt * BM);
+                            tma_load_2d(a + A_BYTES, &tm_wt, &sh.full[s], (kb + q) * BK, un.n0);
+                        }
+                        ++it;
+                    }
                 }
             }
             // Never leave the CTA with copies still landing in its shared memory.
@@ -318,7 +341,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtenso
             int local = 0;
             bool ok = true;
             for (int u = blockIdx.x; ok && u < p.n_units; u += gridDim.x, ++local) {
-                const uint32_t IDESC = unit_of<BN, EPI == kResidual>(p, u).width == BN ? IDESC_WHOLE : IDESC_TAIL;
+                const bool whole = unit_of<BN, EPI == kResidual>(p, u).width == BN;
                 const int buf = local & 1;
                 // The epilogue must have read this accumulator out (two tiles ago) before it is overwritten.
                 if (local >= 2 && !mbar_wait(&sh.acc_empty[buf], ((local >> 1) - 1) & 1, p.err, abort)) {
@@ -327,20 +350,43 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtenso
                 }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem + static_cast<uint32_t>(buf * BN);
-                for (int kb = 0; kb < p.kblocks; ++kb, ++it) {
-                    const int s = static_cast<int>(it % STAGES);
-                    if (!mbar_wait(&sh.full[s], (it / STAGES) & 1, p.err, abort)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    const uint32_t a_addr = base + static_cast<uint32_t>(s * STAGE_BYTES);
-                    const uint32_t b_addr = a_addr + A_BYTES;
+                if (whole) {
+                    for (int kb = 0; kb < p.kblocks; ++kb, ++it) {
+                        const int s = static_cast<int>(it % STAGES);
+                        if (!mbar_wait(&sh.full[s], (it / STAGES) & 1, p.err, abort)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        const uint32_t a_addr = base + static_cast<uint32_t>(s * STAGE_BYTES);
+                        const uint32_t b_addr = a_addr + A_BYTES;
 #pragma unroll
-                    for (int kk = 0; kk < BK / 16; ++kk)
-                        umma_ss(d_tmem, sw128_desc(a_addr + kk * 32, 16, 1024), sw128_desc(b_addr + kk * 32, 16, 1024),
-                                IDESC, (kb > 0 || kk > 0) ? 1u : 0u);
-                    umma_commit(&sh.empty[s]);
+                        for (int kk = 0; kk < BK / 16; ++kk)
+                            umma_ss(d_tmem, sw128_desc(a_addr + kk * 32, 16, 1024),
+                                    sw128_desc(b_addr + kk * 32, 16, 1024), IDESC_WHOLE, (kb > 0 || kk > 0) ? 1u : 0u);
+                        umma_commit(&sh.empty[s]);
+                    }
+                } else {
+                    for (int kb = 0; kb < p.kblocks; kb += TAIL_PER_STAGE, ++it) {
+                        const int s = static_cast<int>(it % STAGES);
+                        if (!mbar_wait(&sh.full[s], (it / STAGES) & 1, p.err, abort)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        const int nk = kb + TAIL_PER_STAGE <= p.kblocks ? TAIL_PER_STAGE : p.kblocks - kb;
+                        for (int q = 0; q < nk; ++q) {
+                            const uint32_t a_addr =
+                                base + static_cast<uint32_t>(s * STAGE_BYTES + q * TAIL_KB_BYTES);
+                            const uint32_t b_addr = a_addr + A_BYTES;
+#pragma unroll
+                            for (int kk = 0; kk < BK / 16; ++kk)
+                                umma_ss(d_tmem, sw128_desc(a_addr + kk * 32, 16, 1024),
+                                        sw128_desc(b_addr + kk * 32, 16, 1024), IDESC_TAIL,
+                                        (kb + q > 0 || kk > 0) ? 1u : 0u);
+                        }
+                        umma_commit(&sh.empty[s]);
+                    }
                 }
                 if (!ok) break;
                 umma_commit(&sh.acc_full[buf]);
