@@ -73,14 +73,10 @@ constexpr float kRescaleThreshold = 8.0f;   // log2 units: O is rescaled only wh
 #ifndef GQA_PREP_POS
 #define GQA_PREP_POS 8
 #endif
-#ifndef GQA_PREP_UNROLL
-#define GQA_PREP_UNROLL 8
-#endif
 #ifndef GQA_PREP_MIN_CTAS
 #define GQA_PREP_MIN_CTAS 2
 #endif
 constexpr int PREP_POS = GQA_PREP_POS;          // positions per CTA of the prep kernel
-constexpr int PREP_UNROLL = GQA_PREP_UNROLL;    // work items per thread in flight
 constexpr int PREP_THREADS = 256;
 
 struct Params {
@@ -124,6 +120,10 @@ struct alignas(8) Shared {
 // ---------------------------------------------------------------------------------------------
 // prep_kernel: for positions [p0, p0+PREP_POS): the cos/sin table, then every Q and K row at those
 // positions rotated into Q' [B*h_q, L, D] and K' [B*h_kv, L, D].
+// Thread t owns 16-byte chunk c = t % CH of each half row (8 rotation pairs: dims 8c.. and their partners
+// 8c + D/2..) and walks the rows (b, head) r0, r0 + RPP, ... (r0 = t / CH), each at all PREP_POS positions
+// of the block: one row per round, its loads issued together.  The pass issues few instructions per byte
+// (one division per row, 16-byte table reads, paired fp32 rotation), which is what bounds it.
 template <int D>
 __global__ void __launch_bounds__(PREP_THREADS, GQA_PREP_MIN_CTAS) prep_kernel(const __nv_bfloat16* __restrict__ q,
                                                             const __nv_bfloat16* __restrict__ k,
@@ -131,85 +131,89 @@ __global__ void __launch_bounds__(PREP_THREADS, GQA_PREP_MIN_CTAS) prep_kernel(c
                                                             __nv_bfloat16* __restrict__ kr, int B, int L,
                                                             int h_q, int h_kv, RopeSpec rope, float mscale) {
     constexpr int H = D / 2;
-    constexpr int CH = D / 16;   // one work item = 8 pairs: a 16-byte chunk of the first half + its partner
-    // Table row pp holds the D/2 (cos, sin) pairs of position p0 + pp, one padding slot after every 8, so
-    // the 8 chunks of a row (read by 8 neighbouring lanes) fall in 8 different shared-memory banks.
-    constexpr int TROW = H + H / 8;
-    __shared__ float2 tab[PREP_POS * TROW];
+    constexpr int CH = D / 16;                 // 16-byte chunks of a half row
+    constexpr int RPP = PREP_THREADS / CH;     // rows per round of the block
+    // Table row pp: (cos f_i, cos f_i+1, sin f_i, sin f_i+1) of position p0 + pp for i = 2j, as float4 j, with
+    // one float4 of padding after every 4, so the CH lanes reading the 4 float4 of their chunks hit
+    // distinct banks (lanes of the same chunk read the same address).
+    constexpr int TROW4 = H / 2 + H / 8;
+    __shared__ float4 tab[PREP_POS * TROW4];
     // The attention kernel launched after this one may be scheduled now; it waits for this grid's
     // results (griddepcontrol.wait) before reading Q' or K'.
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     __shared__ double finv[H];
     const int p0 = blockIdx.x * PREP_POS;
     const int heads = h_q + h_kv;
-    const int bh_n = B * heads;
-    const int items = bh_n * PREP_POS * CH;   // < 2^31: B * (h_q + h_kv) is checked on the host
+    const int bh_n = B * heads;   // B * (h_q + h_kv) < 2^31 is checked on the host
+    const int c = threadIdx.x % CH;
+    const int r0 = threadIdx.x / CH;
+    const int np = L - p0 < PREP_POS ? L - p0 : PREP_POS;   // positions of this block (the last may be short)
 
-    // PREP_UNROLL items per thread per round, loads first, so each thread keeps several 32-byte reads in
-    // flight (the pass is bandwidth bound); the first round's loads are issued before the table is built.
-    uint4 x[PREP_UNROLL], y[PREP_UNROLL];
-    __nv_bfloat16* dst[PREP_UNROLL];
-    int cc[PREP_UNROLL], ppp[PREP_UNROLL];
-    auto load_round = [&](int base) {
+    uint4 x[PREP_POS], y[PREP_POS];
+    __nv_bfloat16* dst = nullptr;   // row pp of the current round's destination: dst + pp * D
+    auto load_row = [&](int bh) {
+        const int b = bh / heads, h = bh - (bh / heads) * heads;
+        const __nv_bfloat16* src;
+        int64_t stride;
+        if (h < h_q) {
+            src = q + ((static_cast<int64_t>(b) * L + p0) * h_q + h) * D;
+            stride = static_cast<int64_t>(h_q) * D;
+            dst = qr + ((static_cast<int64_t>(b) * h_q + h) * L + p0) * D;
+        } else {
+            src = k + ((static_cast<int64_t>(b) * L + p0) * h_kv + (h - h_q)) * D;
+            stride = static_cast<int64_t>(h_kv) * D;
+            dst = kr + ((static_cast<int64_t>(b) * h_kv + (h - h_q)) * L + p0) * D;
+        }
 #pragma unroll
-        for (int uidx = 0; uidx < PREP_UNROLL; ++uidx) {
-            const int e = base + uidx * static_cast<int>(blockDim.x);
-            // item e: chunk fastest, then the row (b, head), then the position, so a warp works on 4 rows
-            // of one position and its table reads are 8 distinct addresses, each broadcast to 4 lanes.
-            dst[uidx] = nullptr;
-            cc[uidx] = e % CH;
-            const int bh = (e / CH) % bh_n;
-            ppp[uidx] = e / (CH * bh_n);
-            const int pos = p0 + ppp[uidx];
-            if (e >= items || pos >= L) continue;
-            const int b = bh / heads, h = bh % heads;
-            const __nv_bfloat16* src;
-            if (h < h_q) {
-                src = q + ((static_cast<int64_t>(b) * L + pos) * h_q + h) * D;
-                dst[uidx] = qr + ((static_cast<int64_t>(b) * h_q + h) * L + pos) * D;
-            } else {
-                src = k + ((static_cast<int64_t>(b) * L + pos) * h_kv + (h - h_q)) * D;
-                dst[uidx] = kr + ((static_cast<int64_t>(b) * h_kv + (h - h_q)) * L + pos) * D;
+        for (int pp = 0; pp < PREP_POS; ++pp) {
+            if (pp < np) {
+                const uint4* row = reinterpret_cast<const uint4*>(src + pp * stride);
+                x[pp] = __ldg(row + c);
+                y[pp] = __ldg(row + c + CH);
             }
-            x[uidx] = __ldg(reinterpret_cast<const uint4*>(src) + cc[uidx]);
-            y[uidx] = __ldg(reinterpret_cast<const uint4*>(src) + cc[uidx] + CH);
         }
     };
-    int base = threadIdx.x;
-    load_round(base);
+    // The first round's loads go out before the table is built.
+    if (r0 < bh_n) load_row(r0);
 
     // theta^(-2i/D) = 2^(-(2i/D) * log2(theta)), scaled under YaRN
     for (int i = threadIdx.x; i < H; i += blockDim.x) finv[i] = rope_freq(i, D, rope);
     __syncthreads();
-    for (int e = threadIdx.x; e < PREP_POS * H; e += blockDim.x) {
-        const int pp = e / H, i = e % H;
-        float c = 1.f, s = 0.f;
-        if (p0 + pp < L) rope_cossin(static_cast<double>(p0 + pp), finv[i], c, s);
-        tab[pp * TROW + i + i / 8] = make_float2(c * mscale, s * mscale);   // YaRN temperature on Q and K
+    for (int e = threadIdx.x; e < PREP_POS * (H / 2); e += blockDim.x) {
+        const int pp = e / (H / 2), j = e % (H / 2);
+        float c0 = 1.f, s0 = 0.f, c1 = 1.f, s1 = 0.f;
+        if (pp < np) {
+            rope_cossin(static_cast<double>(p0 + pp), finv[2 * j], c0, s0);
+            rope_cossin(static_cast<double>(p0 + pp), finv[2 * j + 1], c1, s1);
+        }
+        // YaRN temperature on Q and K (1 without scaling)
+        tab[pp * TROW4 + j + j / 4] = make_float4(c0 * mscale, c1 * mscale, s0 * mscale, s1 * mscale);
     }
     __syncthreads();
 
-    for (; base < items; base += PREP_UNROLL * static_cast<int>(blockDim.x)) {
-        if (base != threadIdx.x) load_round(base);
+    const uint64_t neg1 = f2_pack(-1.f, -1.f);
+    for (int bh = r0; bh < bh_n; bh += RPP) {
+        if (bh != r0) load_row(bh);
 #pragma unroll
-        for (int uidx = 0; uidx < PREP_UNROLL; ++uidx) {
-            if (dst[uidx] == nullptr) continue;
-            const int c = cc[uidx], pp = ppp[uidx];
-            const uint32_t xs[4] = {x[uidx].x, x[uidx].y, x[uidx].z, x[uidx].w};
-            const uint32_t ys[4] = {y[uidx].x, y[uidx].y, y[uidx].z, y[uidx].w};
+        for (int pp = 0; pp < PREP_POS; ++pp) {
+            if (pp >= np) continue;
+            const uint32_t xs[4] = {x[pp].x, x[pp].y, x[pp].z, x[pp].w};
+            const uint32_t ys[4] = {y[pp].x, y[pp].y, y[pp].z, y[pp].w};
             uint32_t xo[4], yo[4];
 #pragma unroll
             for (int w = 0; w < 4; ++w) {
-                const float2 c0 = tab[pp * TROW + 9 * c + 2 * w];       // i = 8c + 2w, padded
-                const float2 c1 = tab[pp * TROW + 9 * c + 2 * w + 1];
-                float a0, b0, a1, b1;
-                rope_rotate(bf16lo_to_f32(xs[w]), bf16lo_to_f32(ys[w]), c0.x, c0.y, a0, b0);
-                rope_rotate(bf16hi_to_f32(xs[w]), bf16hi_to_f32(ys[w]), c1.x, c1.y, a1, b1);
-                xo[w] = pack_bf16x2(a0, a1);
-                yo[w] = pack_bf16x2(b0, b1);
+                const float4 t = tab[pp * TROW4 + 5 * c + w];   // pairs i = 8c + 2w, +1
+                const uint64_t cs = f2_pack(t.x, t.y), sn = f2_pack(t.z, t.w);
+                const uint64_t X = f2_from_bf16x2(xs[w]), Y = f2_from_bf16x2(ys[w]);
+                // x' = fma(x, cos, -(y sin)), y' = fma(y, cos, x sin): the scalar rotation, two pairs at once
+                const uint64_t xr = f2_fma(X, cs, f2_mul(f2_mul(Y, sn), neg1));
+                const uint64_t yr = f2_fma(Y, cs, f2_mul(X, sn));
+                xo[w] = f2_to_bf16x2(xr);
+                yo[w] = f2_to_bf16x2(yr);
             }
-            reinterpret_cast<uint4*>(dst[uidx])[c] = make_uint4(xo[0], xo[1], xo[2], xo[3]);
-            reinterpret_cast<uint4*>(dst[uidx])[c + CH] = make_uint4(yo[0], yo[1], yo[2], yo[3]);
+            uint4* out = reinterpret_cast<uint4*>(dst + pp * D);
+            out[c] = make_uint4(xo[0], xo[1], xo[2], xo[3]);
+            out[c + CH] = make_uint4(yo[0], yo[1], yo[2], yo[3]);
         }
     }
 }
