@@ -1,22 +1,24 @@
 #!/usr/bin/env python
 """Benchmark of the GQA hot path on B200: prefill TFLOP/s and decode KV-cache GB/s.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference|flashinfer]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
     torchrun --nproc-per-node N bench.py --gpus N ...      (one process per GPU)
 
-One step is one pass of the whole hot path: a causal prefill over the Qwen2-7B-shaped workload
-(B=1, L=4096, 28/4 heads, d=128) followed by one decode step over the Qwen2-7B-shaped decode
-workload (B=64 sequences, cache lengths uniform in [1, 32768]).  The headline `value` is the
-prefill's causal-effective TFLOP/s (4*B*h_q*d*L(L+1)/2 per step, summed over ranks, divided by
-the slowest rank's device time); the decode step is reported beside it in GB/s of KV cache.
-Inputs are synthetic (seeded N(0,1) bf16, drawn on the device) and resident in HBM when the
-timed region starts; the L2 is flushed (a 256 MiB write) before every prefill, and the decode
-cache (~2.1 GB) is far larger than L2.  Each rank of an N-GPU run processes its own copy of
-the workload (independent batches, no collective on the data path: weak scaling).
+One step is one pass of the whole hot path: a causal prefill over the largest single-GPU prefill
+workload, Qwen2-7B-shaped long context (B=1, L=32768, 28/4 heads, d=128), followed by one decode step
+over the Qwen2-7B-shaped decode workload (B=64 sequences, cache lengths uniform in [1, 32768]).  The
+headline `value` is the prefill's causal-effective TFLOP/s (4*B*h_q*d*L(L+1)/2 per step, summed over
+ranks, divided by the slowest rank's device time); the decode step is reported beside it in GB/s of KV
+cache.  The other prefill workloads (Qwen2-0.5B L=128, Qwen2-7B L=4096, Qwen2-72B B=4 L=8192) are timed
+the same way after the headline and reported under `configs`, each with its step and kernel times, its
+roofline fraction and a CPU-oracle sample.  Inputs are synthetic (seeded N(0,1) bf16, drawn on the
+device) and resident in HBM when the timed region starts; the L2 is flushed (a 256 MiB write) before
+every prefill, and the decode cache (~2.1 GB) is far larger than L2.  Each rank of an N-GPU run
+processes its own copy of the workload (independent batches, no collective on the data path: weak
+scaling).
 
-`--impl reference` times the plain fp64 CPU oracle (the only reference that exists for this
-method) on a bounded sample of the same prefill workload, on the host cores of rank 0.
-`--impl flashinfer` times installed library attention kernels on the prefill workload, for context.
+`--impl reference` times the plain fp64 CPU oracle (the only reference that exists for this method) on a
+bounded sample of the same prefill workload, on the host cores of rank 0.
 """
 from __future__ import annotations
 
@@ -41,7 +43,9 @@ import torch  # noqa: E402
 import gqa_inputs as gi  # noqa: E402
 
 METRIC = "GQA prefill TFLOP/s & decode KV GB/s, as % of B200 tensor/HBM peak"
-PREFILL_WORKLOAD = "qwen2-7b-prefill-L4096"
+PREFILL_WORKLOAD = "qwen2-7b-prefill-L32768"   # the largest prefill workload that fits one GPU
+# The other prefill workloads, each timed after the headline and reported under `configs`.
+CONFIG_WORKLOADS = ("qwen2-0.5b-prefill-L128", "qwen2-7b-prefill-L4096", "qwen2-72b-prefill-B4-L8192")
 DECODE_WORKLOAD = "qwen2-7b-decode-B64"
 FLUSH_BYTES = 256 << 20
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -205,32 +209,40 @@ def blas_threads() -> int:
     return os.cpu_count() or 1
 
 
+ORACLE_ROW_BLOCK = 1024   # query rows per CPU-oracle sample (bounds one sample to about a second at L=32768)
+
+
 def oracle_prefill_sample(w, budget_s: float, max_steps: int | None = None):
-    """Time the fp64 oracle on one-head slices of the prefill workload (heads in turn)."""
+    """Time the fp64 oracle on samples of the prefill workload: one query head of batch row 0 and a block
+    of up to ORACLE_ROW_BLOCK query rows against all keys before them, the heaviest (last) block first,
+    then the next head, and so on.  Returns the causal-effective FLOP of each sample and its seconds."""
     from oracle import gqa_ref as R
     q, k, v = gi.prefill_inputs(w)
-    per_head = prefill_flops(w.with_(B=1, h_q=1, h_kv=1))
-    times, t0 = [], time.perf_counter()
-    t = 0
+    blocks = [(r0, min(w.L, r0 + ORACLE_ROW_BLOCK)) for r0 in range(0, w.L, ORACLE_ROW_BLOCK)][::-1]
+    flops, times, t0, i = [], [], time.perf_counter(), 0
     while True:
-        u = t // w.g
+        t = (i // len(blocks)) % w.h_q
+        r0, r1 = blocks[i % len(blocks)]
+        rows = list(range(r0, r1))
         a = time.perf_counter()
-        R.prefill_ref(q[:1, :, t:t + 1], k[:1, :, u:u + 1], v[:1, :, u:u + 1], w.theta)
+        R.prefill_rows_ref(q, k, v, w.theta, 0, t, rows)
         times.append(time.perf_counter() - a)
-        t = (t + 1) % w.h_q
+        flops.append(4.0 * w.d * sum(r + 1 for r in rows))   # each row r sees keys 0..r
+        i += 1
         if max_steps is not None and len(times) >= max_steps:
             break
         if max_steps is None and time.perf_counter() - t0 >= budget_s:
             break
-    return per_head, times
+    return flops, times
 
 
-def cpu_baseline(w) -> dict:
-    per_head, times = oracle_prefill_sample(w, budget_s=12.0)
-    return {"value": per_head * len(times) / sum(times) / 1e12, "unit": "TFLOP/s", "cores": blas_threads(),
+def cpu_baseline(w, budget_s: float = 12.0) -> dict:
+    flops, times = oracle_prefill_sample(w, budget_s=budget_s)
+    return {"value": sum(flops) / sum(times) / 1e12, "unit": "TFLOP/s", "cores": blas_threads(),
             "kind": "oracle",
-            "sample": f"fp64 NumPy oracle, {len(times)} single-head slices (b=0, L={w.L}, d={w.d}) of the "
-                      f"{w.name} workload, {sum(times):.1f} s of host time"}
+            "sample": f"fp64 NumPy oracle, {len(times)} samples of one query head x up to {ORACLE_ROW_BLOCK} query "
+                      f"rows (b=0, L={w.L}, d={w.d}, heaviest rows first) of the {w.name} workload, "
+                      f"{sum(times):.1f} s of host time"}
 
 
 def bench_config(wp, wd):
@@ -244,91 +256,22 @@ def run_reference(args):
     rank, _, world = dist_env()
     if rank != 0:
         return 0
-    w = gi.BY_NAME[PREFILL_WORKLOAD]
-    per_head, times = oracle_prefill_sample(w, 0.0, max_steps=args.warmup + args.steps)
+    w = gi.BY_NAME[args.prefill_workload]
+    flops, times = oracle_prefill_sample(w, 0.0, max_steps=args.warmup + args.steps)
     timed = times[args.warmup:]
-    value = per_head * len(timed) / sum(timed) / 1e12
+    value = sum(flops[args.warmup:]) / sum(timed) / 1e12
     line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": 1e3 * sum(timed) / len(timed), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": dict(bench_config(w, gi.BY_NAME[DECODE_WORKLOAD]),
-                           step="one query head of batch row 0 through the fp64 oracle on the host"),
+                           step=f"one query head of batch row 0 x up to {ORACLE_ROW_BLOCK} query rows through "
+                                "the fp64 oracle on the host"),
             "impl": "reference",
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
-                             "sample": f"{len(timed)} single-head slices of {w.name}"},
+                             "sample": f"{len(timed)} samples of one query head x up to {ORACLE_ROW_BLOCK} "
+                                       f"query rows of {w.name}"},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
-    return 0
-
-
-# ------------------------------------------------------------------------------ library context arm
-def run_library(args):
-    """Time flashinfer's Blackwell attention kernels on the prefill workload (context, not a target).
-
-    Plain causal GQA attention on the same shape, inputs, FLOP count and L2 flush as the prefill of
-    `--impl ours`, without RoPE: compare its TFLOP/s with the `roofline.achieved` of our attention
-    kernel.  Backends: "trtllm-gen" (TensorRT-LLM FMHA, precompiled), "cutlass" (CUTLASS sm100 FMHA,
-    compiled on first use, about two minutes), "cute-dsl" (CuTe DSL kernel).  Rank 0 only.
-    """
-    rank, local, _ = dist_env()
-    if rank != 0:
-        return 0
-    import flashinfer
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    w = gi.BY_NAME[args.prefill_workload]
-    B, L, hq, hkv, d = w.B, w.L, w.h_q, w.h_kv, w.d
-    q4, k4, v4 = gi.prefill_inputs(w, device=str(dev))
-    q, k, v = q4.reshape(B * L, hq, d), k4.reshape(B * L, hkv, d), v4.reshape(B * L, hkv, d)
-    indptr = torch.arange(0, (B + 1) * L, L, dtype=torch.int32, device=dev)
-    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
-    fl = prefill_flops(w)
-    results = {}
-    for backend in args.library_backends.split(","):
-        ws = torch.zeros(256 << 20, dtype=torch.uint8, device=dev)
-        if backend == "trtllm-gen":
-            page = 64
-            npg = (L + page - 1) // page
-            pad = npg * page - L
-            def paged(x):
-                x = torch.nn.functional.pad(x.reshape(B, L, hkv, d), (0, 0, 0, 0, 0, pad))
-                return x.view(B, npg, page, hkv, d).permute(0, 1, 3, 2, 4).reshape(B * npg, hkv, page, d).contiguous()
-            kc, vc = paged(k), paged(v)
-            bt = torch.arange(B * npg, dtype=torch.int32, device=dev).view(B, npg)
-            sl = torch.full((B,), L, dtype=torch.int32, device=dev)
-            o = torch.empty_like(q)
-            fn = lambda: flashinfer.prefill.trtllm_batch_context_with_kv_cache(
-                q, (kc, vc), ws, bt, sl, L, L, 1.0 / d ** 0.5, 1.0, B, indptr, indptr, out=o,
-                kv_layout="HND", causal=True)
-        else:
-            wr = flashinfer.BatchPrefillWithRaggedKVCacheWrapper(ws, "NHD", backend=backend)
-            wr.plan(indptr, indptr, hq, hkv, d, causal=True, q_data_type=torch.bfloat16,
-                    kv_data_type=torch.bfloat16)
-            fn = lambda: wr.run(q, k, v)
-        for _ in range(args.warmup):
-            fn()
-        ms = []
-        for _ in range(args.steps):
-            flush.zero_()
-            a, b = ev(), ev()
-            a.record()
-            fn()
-            b.record()
-            torch.cuda.synchronize()
-            ms.append(a.elapsed_time(b))
-        mean = sum(ms) / len(ms)
-        results[backend] = {"ms_per_launch": mean, "tflops": fl / mean / 1e9}
-    best = max(results, key=lambda b_: results[b_]["tflops"])
-    peaks, src = load_peaks()
-    line = {"metric": METRIC, "value": results[best]["tflops"], "unit": "TFLOP/s", "n_gpus": 1,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": results[best]["ms_per_launch"],
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-            "data": "synthetic", "config": dict(bench_config(w, gi.BY_NAME[DECODE_WORKLOAD]),
-                                                 step="attention kernel only, no RoPE, L2 flushed before each launch"),
-            "impl": "flashinfer", "flashinfer_version": flashinfer.__version__, "best_backend": best,
-            "frac_of_bf16_peak": results[best]["tflops"] / peaks["bf16_tflops"], "peak_source": src,
-            "backends": results}
-    print(json.dumps(clean(line)), flush=True)
     return 0
 
 
@@ -339,9 +282,63 @@ def ev():
     return e
 
 
+def measure_prefill(G, w, K: int, W: int, flush, dev):
+    """Time gqa_prefill on workload w: W warm-up steps, then K headline steps (no per-kernel events, so
+    the attention kernel stays a programmatic dependent of the rotation pass) interleaved with K steps
+    that record events around the attention kernel alone; the L2 is flushed before every step.
+    Returns (mean step ms, max over ranks; mean attention-kernel ms on this rank)."""
+    q, k, v = gi.prefill_inputs(w, device=str(dev))
+    out = torch.empty_like(q)
+
+    def step(e, inner):
+        flush.zero_()
+        e[0].record()
+        if inner:
+            G.set_timing_events(e[1], e[2])
+        G.prefill(q, k, v, theta=w.theta, out=out)
+        if inner:
+            G.set_timing_events(None, None)
+        e[3].record()
+
+    for _ in range(W):
+        step([ev() for _ in range(4)], False)
+    evs = [[ev() for _ in range(4)] for _ in range(K)]
+    kevs = [[ev() for _ in range(4)] for _ in range(K)]
+    torch.cuda.synchronize()
+    barrier()
+    for i in range(K):
+        step(evs[i], False)
+        step(kevs[i], True)
+    torch.cuda.synchronize()
+    barrier()
+    if G.last_error() != 0:
+        raise RuntimeError(f"device error while timing {w.name}")
+    step_ms = reduce_max(sum(e[0].elapsed_time(e[3]) for e in evs) / K, dev)
+    attn_ms = sum(e[1].elapsed_time(e[2]) for e in kevs) / K
+    del q, k, v, out
+    return step_ms, attn_ms
+
+
+def config_entry(w, *, world, step_ms, attn_ms, peaks, peak_src, cpu_base):
+    """The `configs` entry of one prefill workload from its measured step and kernel times (ms)."""
+    fl = prefill_flops(w)
+    step_t = fl / (step_ms * 1e-3) / 1e12
+    ach = fl / (attn_ms * 1e-3) / 1e12
+    return {"workload": w.desc, "B": w.B, "L": w.L, "h_q": w.h_q, "h_kv": w.h_kv, "d": w.d,
+            "value": world * step_t, "unit": "TFLOP/s", "ms_per_step": step_ms,
+            "step_frac": step_t / peaks["bf16_tflops"],
+            "kernel_ms_per_launch": attn_ms,
+            "roofline": {"kernel": "attn_kernel (prefill)", "bound": "tensor", "achieved": ach,
+                         "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": ach / peaks["bf16_tflops"],
+                         "peak_source": f"{peak_src} bf16 dense (burst)",
+                         "traffic": profile_traffic("attn_kernel", w.name),
+                         "algorithmic_flops_per_launch": fl, "ms_per_launch": attn_ms},
+            "cpu_baseline": cpu_base}
+
+
 def build_line(*, world, K, W, only, do_p, do_d, wp, wd, value_tflops, pre_mean, attn_mean, dec_mean, split_mean,
                total_rows, page, peaks, peak_src, cpu_base, e2e_pre, e2e_dec, pre_io, dec_io, qkv_line, clocks,
-               t_wall):
+               t_wall, configs=None):
     """The JSON line of the `ours` arm from the measured numbers (no device work, so the CPU tests cover it).
     Times in ms; pre_io / dec_io = (host->device, device->host) bytes of one end-to-end prefill / decode
     step; a leg that did not run carries NaN, which clean() turns into null."""
@@ -377,7 +374,8 @@ def build_line(*, world, K, W, only, do_p, do_d, wp, wd, value_tflops, pre_mean,
         "only": only,
         "e2e": {"value": world * fl / (e2e_pre * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "h2d_bytes_per_step": pre_io[0], "d2h_bytes_per_step": pre_io[1]},
-        "gpu_launches": (2 * do_p + 3 * do_d) * 2 * K + (6 * K if qkv_line else 0),
+        "gpu_launches": (2 * do_p + 3 * do_d) * 2 * K + (6 * K if qkv_line else 0)
+                        + 2 * 2 * K * sum(1 for n in (configs or {}) if n != wp.name),
         "qkv": qkv_line,
         "clocks": clocks,
         "decode": {
@@ -399,6 +397,10 @@ def build_line(*, world, K, W, only, do_p, do_d, wp, wd, value_tflops, pre_mean,
         },
         "wall_s_timed_region": t_wall,
         "impl": "ours",
+        # every prefill workload: the headline's own figures, then the others timed after it
+        "configs": dict({wp.name: config_entry(wp, world=world, step_ms=pre_mean, attn_ms=attn_mean, peaks=peaks,
+                                               peak_src=peak_src, cpu_base=cpu_base)} if do_p else {},
+                        **(configs or {})),
     }
     if not do_p:   # --only decode: the line carries the decode half alone
         line["roofline"] = line["e2e"] = line["cpu_baseline"] = None
@@ -621,6 +623,18 @@ def run_ours(args):
         del xq, wqkv, bqkv, qo, w_o, x_in, y_out
 
     peaks, peak_src = load_peaks()
+    # ---- the other prefill workloads, one after another (each rank its own copy), each with its own
+    # step and kernel times, roofline fraction and (rank 0 of a 1-GPU run) a bounded CPU-oracle sample
+    configs = {}
+    names = [] if args.configs in ("", "none") or not do_p else [n for n in args.configs.split(",") if n != wp.name]
+    for name in names:
+        wc = gi.BY_NAME[name]
+        with ClockSampler(local) as c_clk:
+            c_step, c_attn = measure_prefill(G, wc, K, W, flush, dev)
+        c_cpu = cpu_baseline(wc, budget_s=4.0) if (rank == 0 and world == 1 and not args.no_cpu_baseline) else None
+        configs[name] = config_entry(wc, world=world, step_ms=c_step, attn_ms=c_attn, peaks=peaks,
+                                     peak_src=peak_src, cpu_base=c_cpu)
+        configs[name]["clocks"] = c_clk.summary()
     line = None
     if rank == 0:
         line = build_line(
@@ -631,7 +645,7 @@ def run_ours(args):
             e2e_pre=e2e_pre, e2e_dec=e2e_dec,
             pre_io=(sum(x.numel() * x.element_size() for x in (q, k, v)), out.numel() * out.element_size()),
             dec_io=(qd.numel() * 2 + s.numel() * 4 + (table.numel() * 4 if page else 0), outd.numel() * 2),
-            qkv_line=qkv_line, clocks=sampler.summary(), t_wall=t_wall)
+            qkv_line=qkv_line, clocks=sampler.summary(), t_wall=t_wall, configs=configs)
     if torch.distributed.is_initialized():
         barrier()
         torch.distributed.destroy_process_group()
@@ -645,17 +659,17 @@ def main(argv=None):
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--impl", choices=["ours", "reference", "flashinfer"], default="ours",
-                    help="ours: the CUDA path; reference: the fp64 oracle on the host; flashinfer: library "
-                         "attention kernels on the prefill workload, for context")
-    ap.add_argument("--library-backends", default="trtllm-gen",
-                    help="flashinfer backends timed by --impl flashinfer (comma list of trtllm-gen, cutlass, cute-dsl)")
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours",
+                    help="ours: the CUDA path; reference: the fp64 oracle on the host")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the host oracle timing")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffer) leg")
     ap.add_argument("--only", choices=["prefill", "decode"], default=None,
                     help="run one half of the step only (profiling; the line then carries that half)")
     ap.add_argument("--prefill-workload", default=PREFILL_WORKLOAD, choices=[w.name for w in gi.WORKLOADS if w.kind == "prefill"],
-                    help="prefill workload of the step (default: the Qwen2-7B L=4096 headline workload)")
+                    help="prefill workload of the step (default: the Qwen2-7B L=32768 headline workload)")
+    ap.add_argument("--configs", default=",".join(CONFIG_WORKLOADS),
+                    help="comma list of further prefill workloads timed after the headline and reported under "
+                         "`configs` ('none' for none)")
     ap.add_argument("--no-qkv", action="store_true", help="skip the fused QKV projection leg")
     ap.add_argument("--decode-page-size", type=int, default=None,
                     help="decode through gqa_decode_paged, the cache in pages of this many rows")
@@ -666,8 +680,6 @@ def main(argv=None):
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
         return run_reference(args)
-    if args.impl == "flashinfer":
-        return run_library(args)
     return run_ours(args)
 
 

@@ -581,8 +581,8 @@ int launch_decode(DeviceState* st, const void* q, const void* kc, const void* vc
     // CTAS_PER_SM CTAs of WARPS workers per SM in total, split evenly over the (group, head block) pairs.
     const int G = (CTAS_PER_SM * st->num_sms + groups - 1) / groups;
     const int P = G * WARPS;
-    const size_t off_bytes = (static_cast<size_t>(B + 1) * sizeof(int64_t) + 255) & ~size_t(255);
-    const size_t part_bytes = static_cast<size_t>(P + B) * groups * C::PART * sizeof(float);
+    const size_t off_bytes = ((static_cast<size_t>(B) + 1) * sizeof(int64_t) + 255) & ~size_t(255);
+    const size_t part_bytes = (static_cast<size_t>(P) + static_cast<size_t>(B)) * groups * C::PART * sizeof(float);
     if (!ensure(st->dws, st->dws_bytes, off_bytes + part_bytes)) return GQA_ERR_ALLOC;
 
     Params p;
@@ -645,8 +645,8 @@ int launch_decode_fixed_scratch(DeviceState* st, const void* q, const void* kc, 
     const int groups = h_kv * n_hb;
     const int G = (CTAS_PER_SM * st->num_sms + groups - 1) / groups;
     const int P = G * WARPS;
-    const size_t off_bytes = (static_cast<size_t>(B + 1) * sizeof(int64_t) + 255) & ~size_t(255);
-    const size_t part_bytes = static_cast<size_t>(P + B) * groups * C::PART * sizeof(float);
+    const size_t off_bytes = ((static_cast<size_t>(B) + 1) * sizeof(int64_t) + 255) & ~size_t(255);
+    const size_t part_bytes = (static_cast<size_t>(P) + static_cast<size_t>(B)) * groups * C::PART * sizeof(float);
     if (off_bytes + part_bytes > kFixedScratchBytes) return GQA_ERR_TOO_LARGE;
     const int rc = fixed_scratch_setup(st);
     if (rc != GQA_OK) return rc;

@@ -113,10 +113,11 @@ GQA_API int gqa_set_timing_events(void* start_event, void* stop_event);
  * partials) is a fixed 16 MiB array in the library's device memory, which every GPU that loads the
  * library holds until the process exits.
  *
- * Limit: the scratch needed is 8*(B+1) bytes rounded up to 256, plus
- * (P + B) * h_kv * ceil(g/8) * (16 + 8*d) * 4 bytes, where P = 4 * ceil(2*SMs / (h_kv*ceil(g/8)))
- * (P = 296 for h_kv = 4 on a 148-SM B200: the Qwen2-7B shape fits up to B of about 700).  Larger
- * problems return GQA_ERR_TOO_LARGE and launch nothing.
+ * Limit: the scratch needed is 8*(B+1) bytes rounded up to a multiple of 256, plus
+ * (P + B) * h_kv * ceil(g/8) * (16 + 8*d) * 4 bytes, where P = 4 * ceil(3*SMs / (h_kv*ceil(g/8)))
+ * (3 split CTAs of 4 warps per SM; P = 444 for h_kv = 4, g = 7 on a 148-SM B200, so the Qwen2-7B
+ * shape fits up to B = 563).  The total must not exceed 16 MiB (16777216 bytes); larger problems
+ * return GQA_ERR_TOO_LARGE and launch nothing.
  *
  * The first call on a device looks up the device address of the fixed array (with that device
  * current); make that first call before any stream capture.  All calls on a device share the one

@@ -47,8 +47,10 @@ into independent blocks (each block is still the full materialised product):
      alpha_i; aicoding.csdn.net page, §5.3: a length-dependent rescaling of
      the attention logits).  The pages give neither the ramp's bounds nor
      the rescaling formula; ``Yarn`` takes the published YaRN method's
-     (turn-count bounds 1 and 32, temperature (0.1 ln s + 1)^2): parity
-     partly unpinned.  Pass a ``Yarn`` wherever ``theta`` is taken.
+     (turn-count bounds 1 and 32, temperature (0.1 ln s + 1)^2).  Parity
+     unpinned by the pages for those constants: the pins fix only the
+     form (factor 1 = plain RoPE, fast pairs kept, slow pairs divided by s,
+     logits rescaled).  Pass a ``Yarn`` wherever ``theta`` is taken.
 
 Every function is pinned by ``tests/test_oracle_pins.py`` against closed forms,
 invariants the pages state and a brute-force restatement.

@@ -16,7 +16,7 @@ CONTRACT = ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step
             "impl")
 
 
-def line_for(only, world=1, page=None, qkv=None):
+def line_for(only, world=1, page=None, qkv=None, configs=None):
     do_p, do_d = only in (None, "prefill"), only in (None, "decode")
     wp, wd = gi.BY_NAME[bench.PREFILL_WORKLOAD], gi.BY_NAME[bench.DECODE_WORKLOAD]
     fl = bench.prefill_flops(wp)
@@ -30,7 +30,7 @@ def line_for(only, world=1, page=None, qkv=None):
         cpu_base={"value": 0.03, "unit": "TFLOP/s", "cores": 16, "kind": "oracle", "sample": "s"} if do_p else None,
         e2e_pre=1.3 if do_p else NAN, e2e_dec=0.4 if do_d else NAN, pre_io=(37748736, 29360128),
         dec_io=(459008, 458752), qkv_line=qkv, clocks={"sm_mhz": 1965, "sm_max_mhz": 1965, "reasons": []},
-        t_wall=0.05)
+        t_wall=0.05, configs=configs)
     text = json.dumps(bench.clean(line), allow_nan=False)   # strict JSON: no NaN or inf survives
     return json.loads(text)
 
@@ -76,3 +76,30 @@ def test_whole_job_rates_scale_with_ranks(world):
 def test_paged_layout_is_named():
     d = line_for("decode", page=16)
     assert d["decode"]["layout"].startswith("paged: 16 rows per page")
+
+
+def test_headline_is_the_largest_prefill_workload():
+    prefill = [w for w in gi.WORKLOADS if w.kind == "prefill"]
+    assert bench.PREFILL_WORKLOAD == max(prefill, key=bench.prefill_flops).name
+    assert set(bench.CONFIG_WORKLOADS) | {bench.PREFILL_WORKLOAD} == {w.name for w in prefill}
+
+
+def test_configs_carry_step_kernel_roofline_and_cpu_baseline():
+    cb = {"value": 0.03, "unit": "TFLOP/s", "cores": 16, "kind": "oracle", "sample": "s"}
+    times = {"qwen2-0.5b-prefill-L128": (0.02, 0.012), "qwen2-7b-prefill-L4096": (0.13, 0.115),
+             "qwen2-72b-prefill-B4-L8192": (4.0, 3.8)}
+    configs = {n: bench.config_entry(gi.BY_NAME[n], world=1, step_ms=a, attn_ms=b, peaks=PEAKS,
+                                     peak_src="measured", cpu_base=cb) for n, (a, b) in times.items()}
+    d = line_for(None, configs=configs)
+    assert set(d["configs"]) == set(times) | {bench.PREFILL_WORKLOAD}
+    for n, (a, b) in times.items():
+        c = d["configs"][n]
+        fl = bench.prefill_flops(gi.BY_NAME[n])
+        assert c["ms_per_step"] == a and c["kernel_ms_per_launch"] == b
+        assert math.isclose(c["roofline"]["frac"], fl / (b * 1e-3) / 1e12 / PEAKS["bf16_tflops"])
+        assert math.isclose(c["step_frac"], fl / (a * 1e-3) / 1e12 / PEAKS["bf16_tflops"])
+        assert c["cpu_baseline"]["kind"] == "oracle"
+    head = d["configs"][bench.PREFILL_WORKLOAD]
+    assert math.isclose(head["roofline"]["frac"], d["roofline"]["frac"])
+    # two launches (rotation pass + attention) per step, two kinds of step, K steps, three more workloads
+    assert d["gpu_launches"] == (2 + 3) * 2 * 30 + 3 * 2 * 2 * 30

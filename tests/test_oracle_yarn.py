@@ -3,7 +3,9 @@ f_i / s * alpha_i with a ramp alpha_i from 1 to s; aicoding.csdn.net page, §5.3
 rescaling of the attention logits; §5.5: behaviour within the trained window unchanged).  The ramp bounds
 and the temperature come from the published YaRN method, not the pages: these tests pin what the pages fix
 (factor 1 is plain RoPE; slow pairs are interpolated by s, fast pairs kept; logits rescaled) and the
-method's limits, so parity is only partly pinned."""
+method's limits.  The constants themselves -- the ramp bounds of 1 and 32 turns and the temperature
+0.1 ln s + 1 -- are parity unpinned by the pages: nothing on them fixes those numbers, and the tests that
+mention them are consistency checks of the oracle's own choice."""
 import numpy as np
 import pytest
 
@@ -50,9 +52,13 @@ def test_slow_pairs_at_position_p_turn_like_plain_rope_at_p_over_s():
     np.testing.assert_allclose(a[..., idx], b[..., idx], atol=1e-12)
 
 
-def test_temperature_scales_the_logits_by_mscale_squared():
-    """With a huge original window every pair turns >= 32 times, so no frequency changes and only the
-    temperature remains: attention = softmax(m^2 * plain scores) V."""
+def test_temperature_consistency_logits_scale_by_the_square_of_the_row_factor():
+    """A consistency check, not a pin: the value m = rope_mscale(y) = 0.1 ln s + 1 is the published YaRN
+    method's, which the pages do not give (parity unpinned by the pages), and it is restated here.  What
+    this does check is how the oracle applies it: as a factor on every rotated Q and K row, so that the
+    scores, and only the scores, scale by m^2.  With a huge original window every pair turns >= 32
+    times, so no frequency changes and only the temperature remains: attention = softmax(m^2 * plain
+    scores) V."""
     rng = np.random.default_rng(3)
     L, h_q, h_kv, d = 7, 2, 1, 16
     q, k, v = rng.standard_normal((1, L, h_q, d)), rng.standard_normal((1, L, h_kv, d)), rng.standard_normal((1, L, h_kv, d))
