@@ -35,6 +35,10 @@ into independent blocks (each block is still the full materialised product):
      KV head in fixed-size blocks): the same decode, with position j of
      sequence b read from slot j % page_size of page block_table[b, j //
      page_size].  ``decode_paged_ref`` gathers the rows and applies step 4.
+     ``qkv_append_ref`` is one decode step's projection: the new token's q,
+     and its k, v written into the page slot of position seqlens[b] (the
+     cache grows by the current token each step, aicoding.csdn.net page,
+     §4.1.3 closing paragraph).
   6. QKV projection (aicoding.csdn.net page, §4.1.3 steps 1-3): Q, K, V are
      the hidden states times W_Q, W_K, W_V plus the bias, split into h_q and
      h_kv heads; Q and K are then rotated as in step 1.
@@ -239,12 +243,13 @@ def decode_ref(q, kcache, vcache, seqlens, theta: float, include_self: bool = Fa
     return np.stack(outs, axis=0)
 
 
-def decode_paged_ref(q, kpages, vpages, block_table, seqlens, theta: float, batch_rows=None) -> np.ndarray:
+def decode_paged_ref(q, kpages, vpages, block_table, seqlens, theta: float, batch_rows=None,
+                     include_self: bool = False) -> np.ndarray:
     """Decode step over a paged cache (nxmr.cn page, §2.4: the cache of each KV head kept in blocks).
 
     kpages/vpages [num_pages, page_size, h_kv, d]; block_table [B, max_pages]: position j of sequence b is
     slot j % page_size of page block_table[b, j // page_size].  Gathers each sequence's rows in position
-    order and applies the decode definition of decode_one_ref.
+    order and applies the decode definition of decode_one_ref (``include_self`` as there).
     """
     kp, vp, bt = np.asarray(kpages), np.asarray(vpages), np.asarray(block_table)
     page_size = kp.shape[1]
@@ -254,8 +259,38 @@ def decode_paged_ref(q, kpages, vpages, block_table, seqlens, theta: float, batc
     for b in bs:
         kr = np.stack([kp[bt[b, j // page_size], j % page_size] for j in range(seq[b])])
         vr = np.stack([vp[bt[b, j // page_size], j % page_size] for j in range(seq[b])])
-        outs.append(decode_one_ref(q[b], kr, vr, theta))
+        outs.append(decode_one_ref(q[b], kr, vr, theta, include_self))
     return np.stack(outs, axis=0)
+
+
+def qkv_append_ref(x, w_qkv, b_qkv, h_q: int, h_kv: int, d: int, seqlens, kpages, vpages, block_table):
+    """One decode step's projection and cache append (aicoding.csdn.net page, §4.1.3 steps 1-2 and its
+    closing paragraph: each step appends the current token's K and V to the cache of the h_kv groups;
+    nxmr.cn page, §2.4: that cache kept in pages).
+
+    x [B, d_model] is the new token of each sequence; its projection y = x w_qkv^T + b is split into
+    q [B, h_q, d] and the rows k, v [B, h_kv, d].  The token sits at position p_b = seqlens[b] (the cache
+    length before the append), so k and v go, un-rotated like every cache row, to slot p_b % page_size of
+    page block_table[b, p_b // page_size].  Returns (q float64 [B, h_q, d], un-rotated; the grown key and
+    value pages as float64 copies); the inputs are not modified.
+    """
+    xf, wf = as_f64(x), as_f64(w_qkv)
+    y = xf @ wf.T                                         # [B, (h_q + 2 h_kv) d]
+    if b_qkv is not None:
+        y = y + as_f64(b_qkv)[None, :]
+    B = xf.shape[0]
+    q = y[:, :h_q * d].reshape(B, h_q, d)
+    k = y[:, h_q * d:(h_q + h_kv) * d].reshape(B, h_kv, d)
+    v = y[:, (h_q + h_kv) * d:].reshape(B, h_kv, d)
+    kp, vp = as_f64(kpages).copy(), as_f64(vpages).copy()
+    bt = np.asarray(block_table)
+    page_size = kp.shape[1]
+    for b in range(B):
+        pos = int(np.asarray(seqlens).reshape(-1)[b])
+        page = int(bt[b, pos // page_size])
+        kp[page, pos % page_size] = k[b]
+        vp[page, pos % page_size] = v[b]
+    return q, kp, vp
 
 
 def qkv_rope_ref(x, w_qkv, b_qkv, h_q: int, h_kv: int, d: int, theta: float, positions=None):
