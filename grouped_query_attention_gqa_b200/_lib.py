@@ -47,6 +47,10 @@ def load() -> ctypes.CDLL:
     lib.gqa_decode_paged.restype = i
     lib.gqa_qkv_rope.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f]
     lib.gqa_qkv_rope.restype = i
+    lib.gqa_qkv_append.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i]
+    lib.gqa_qkv_append.restype = i
+    lib.gqa_set_decode_self_in_cache.argtypes = [i]
+    lib.gqa_set_decode_self_in_cache.restype = i
     lib.gqa_prefill_rotated.argtypes = [vp, vp, vp, vp, i, i, i, i, i]
     lib.gqa_prefill_rotated.restype = i
     lib.gqa_out_proj.argtypes = [vp, vp, vp, vp, i, i, i]
@@ -204,6 +208,52 @@ def qkv_rope(x: torch.Tensor, w_qkv: torch.Tensor, b_qkv: torch.Tensor | None, h
     if rc != GQA_OK:
         raise GQAError(rc, "gqa_qkv_rope")
     return qr, kr, k, v
+
+
+def qkv_append(x: torch.Tensor, w_qkv: torch.Tensor, b_qkv: torch.Tensor | None, h_q: int, h_kv: int,
+               seqlens: torch.Tensor, kpages: torch.Tensor, vpages: torch.Tensor, block_table: torch.Tensor,
+               q: torch.Tensor | None = None) -> torch.Tensor:
+    """One decode step's projection and cache append.  x [B, d_model] (the new token of each sequence);
+    w_qkv, b_qkv as for qkv_rope; seqlens int32 [B] (device): each new token's position (the cache length
+    before the append).  Writes the tokens' K (un-rotated) and V into kpages / vpages [num_pages, page_size,
+    h_kv, d] at those positions through block_table int32 [B, max_pages]; returns q [B, h_q, d] (un-rotated)."""
+    if x.dim() != 2 or w_qkv.dim() != 2 or kpages.dim() != 4:
+        raise ValueError("x must be [B, d_model], w_qkv [(h_q + 2 h_kv) d, d_model], kpages [P, page, h_kv, d]")
+    B, dm = x.shape
+    n = w_qkv.shape[0]
+    if n % (h_q + 2 * h_kv) != 0:
+        raise ValueError(f"w_qkv has {n} rows, not a multiple of h_q + 2 h_kv = {h_q + 2 * h_kv}")
+    d = n // (h_q + 2 * h_kv)
+    num_pages, page_size = kpages.shape[:2]
+    _check(x, "x", None)
+    _check(w_qkv, "w_qkv", (n, dm))
+    if b_qkv is not None:
+        _check(b_qkv, "b_qkv", (n,))
+    _check(kpages, "kpages", (num_pages, page_size, h_kv, d))
+    _check(vpages, "vpages", tuple(kpages.shape))
+    _check(seqlens, "seqlens", (B,), dtype=torch.int32)
+    if block_table.dim() != 2 or block_table.shape[0] != B:
+        raise ValueError(f"block_table must be [B={B}, max_pages], got {tuple(block_table.shape)}")
+    _check(block_table, "block_table", None, dtype=torch.int32)
+    if q is None:
+        q = x.new_empty(B, h_q, d)
+    _check(q, "q", (B, h_q, d))
+    with torch.cuda.device(x.device):
+        _stream(x.device)
+        rc = load().gqa_qkv_append(_ptr(x), _ptr(w_qkv), _ptr(b_qkv), _ptr(seqlens), _ptr(q), _ptr(kpages),
+                                   _ptr(vpages), _ptr(block_table), B, dm, h_q, h_kv, d, page_size, num_pages,
+                                   block_table.shape[1])
+    if rc != GQA_OK:
+        raise GQAError(rc, "gqa_qkv_append")
+    return q
+
+
+def set_decode_self_in_cache(on: bool) -> None:
+    """Later decode calls: False (default) -- the query sits at seqlens[b] and attends to the seqlens[b]
+    cached rows; True -- the cache's last row is the query's own, so it sits at seqlens[b] - 1."""
+    rc = load().gqa_set_decode_self_in_cache(1 if on else 0)
+    if rc != GQA_OK:
+        raise GQAError(rc, "gqa_set_decode_self_in_cache")
 
 
 def prefill_rotated(qr: torch.Tensor, kr: torch.Tensor, v: torch.Tensor, out: torch.Tensor | None = None):

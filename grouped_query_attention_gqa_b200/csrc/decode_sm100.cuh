@@ -76,6 +76,7 @@ struct Params {
     const int64_t* off;        // [B + 1] packed row offsets
     float* part;               // [(P + B) * h_kv * n_hb * PART]
     int B, h_q, h_kv, g, n_hb, P;
+    int self_in_cache;         // 1: the cache already holds the query's own row; it sits at seqlens[b] - 1
     float scale_log2;
     RopeSpec rope;             // RoPE base and YaRN scaling (its temperature is in scale_log2)
     int* err;
@@ -192,7 +193,8 @@ __device__ __forceinline__ void rot_step(uint64_t& C, uint64_t& S, uint64_t Cr, 
     C = c2;
 }
 
-template <int D>
+// PAGED: cache rows are read through the block table p.bt (gqa_decode_paged); otherwise packed.
+template <int D, bool PAGED>
 __global__ void __launch_bounds__(WARPS * 32, CTAS_PER_SM) split_kernel(const Params p) {
     using C = Cfg<D>;
     constexpr int H = D / 2;
@@ -251,7 +253,7 @@ __global__ void __launch_bounds__(WARPS * 32, CTAS_PER_SM) split_kernel(const Pa
         // row stays zero and the device error word gets kErrBadPage.
         bool load = i < nvalid;
         int64_t srow = iss.r + i;
-        if (load && p.bt) {
+        if (PAGED && load) {
             const int j = static_cast<int>(srow - p.off[iss.b]);   // position in the sequence (< 2^31)
             const int pi = j / p.page_size;
             const int page = pi < p.max_pages ? p.bt[static_cast<int64_t>(iss.b) * p.max_pages + pi] : -1;
@@ -289,7 +291,8 @@ __global__ void __launch_bounds__(WARPS * 32, CTAS_PER_SM) split_kernel(const Pa
         const int b = cur.b;
         const int64_t seq0 = p.off[b];
         const int64_t seg_end = cur.seg_end;
-        const double qpos = static_cast<double>(p.off[b + 1] - seq0);   // query position = cache length
+        // query position: the cache length, or its last row when that row is the query's own
+        const double qpos = static_cast<double>(p.off[b + 1] - seq0 - p.self_in_cache);
 
         // Q'^T as the B operand: lane holds head t4 of the block, dims 16ks + 2tq + {0,1} (b0) and +8 (b1).
         uint32_t qb[C::KS][2];

@@ -65,11 +65,18 @@ struct DeviceState {
     const void* proj_key[2] = {nullptr, nullptr};
     long long proj_dims[4] = {0, 0, 0, 0};
     CUtensorMap proj_maps[3];
+    const void* app_key[2] = {nullptr, nullptr};
+    long long app_dims[4] = {0, 0, 0, 0};
+    CUtensorMap app_maps[3];
 };
 
 DeviceState g_dev[kMaxDevices];
 cudaStream_t g_stream = nullptr;
 cudaEvent_t g_ev_start = nullptr, g_ev_stop = nullptr;   // optional timing of the main kernel
+
+// Decode query position for every later decode call (gqa_set_decode_self_in_cache): 0 = at seqlens[b],
+// 1 = at seqlens[b] - 1, the cache's last row being the query's own.
+int g_self_in_cache = 0;
 
 // YaRN scaling of RoPE for every later call (gqa_set_rope_scaling); factor 1 = plain RoPE.
 float g_rope_factor = 1.0f;
@@ -531,6 +538,40 @@ int launch_proj(DeviceState* st, const void* attn, const void* w_o, const void* 
     return run_gemm<bn>(st, proj_kernel<bn>, 4u, st->proj_maps, p, true);
 }
 
+// One decode step's projection and cache append: x [B, d_model] (the new token of each sequence) times
+// w_qkv^T + bias; q [B, h_q, D] and the page slots of positions seqlens[b] get the un-rotated heads.
+template <int D>
+int launch_append(DeviceState* st, const void* x, const void* w, const void* bias, const int* seqlens, void* q,
+                  void* kpages, void* vpages, const int* bt, int B, int d_model, int h_q, int h_kv, int page_size,
+                  int num_pages, int max_pages) {
+    using namespace gqa::qkv;
+    const int N = (h_q + 2 * h_kv) * D;
+    const long long mtiles = (static_cast<long long>(B) + BM - 1) / BM;
+    constexpr int bn = 256;
+    if (!gemm_maps(st->app_maps, st->app_key, st->app_dims, x, w, B, d_model, N, bn)) return GQA_ERR_LAUNCH;
+    Params p = {};
+    p.bias = static_cast<const __nv_bfloat16*>(bias);
+    p.qr = static_cast<__nv_bfloat16*>(q);
+    p.k = static_cast<__nv_bfloat16*>(kpages);
+    p.v = static_cast<__nv_bfloat16*>(vpages);
+    p.seqlens = seqlens;
+    p.bt = bt;
+    p.page_size = page_size;
+    p.num_pages = num_pages;
+    p.max_pages = max_pages;
+    p.T = B;
+    p.L = 1;
+    p.N = N;
+    p.h_q = h_q;
+    p.h_kv = h_kv;
+    p.n_ntiles = (N + bn - 1) / bn;
+    if (mtiles * p.n_ntiles > 0x7fffffffLL) return GQA_ERR_DIMS;
+    p.n_tiles = static_cast<int>(mtiles * p.n_ntiles);
+    p.kblocks = (d_model + BK - 1) / BK;
+    p.err = st->err;
+    return run_gemm<bn>(st, append_kernel<D, bn>, D == 128 ? 8u : 16u, st->app_maps, p, false);
+}
+
 // The decode step's three kernels: plan (offsets), split (one partial per piece), combine (merge).
 // Split and combine are programmatic dependents of the kernel before them: their CTAs may start
 // (barrier and RoPE-table set-up) while it drains, and wait for its results with griddepcontrol.wait.
@@ -541,7 +582,9 @@ int launch_decode_chain(const gqa::decode::Params& p, const int* seqlens, int64_
     using C = Cfg<D>;
     const long long cgrid = static_cast<long long>(p.B) * p.h_kv * p.n_hb;
     if (cgrid > 0x7fffffffLL) return GQA_ERR_DIMS;
-    if (cudaFuncSetAttribute(split_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
+    const bool paged = p.bt != nullptr;
+    auto split = paged ? split_kernel<D, true> : split_kernel<D, false>;
+    if (cudaFuncSetAttribute(split, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
         return GQA_ERR_LAUNCH;
     const bool timed = marks && g_ev_start && g_ev_stop;
     cudaLaunchAttribute attr[1];
@@ -559,7 +602,7 @@ int launch_decode_chain(const gqa::decode::Params& p, const int* seqlens, int64_
     cfg.gridDim = dim3(split_grid);
     cfg.blockDim = dim3(WARPS * 32);
     cfg.dynamicSmemBytes = C::SMEM;
-    if (cudaLaunchKernelEx(&cfg, split_kernel<D>, p) != cudaSuccess) return GQA_ERR_LAUNCH;
+    if (cudaLaunchKernelEx(&cfg, split, p) != cudaSuccess) return GQA_ERR_LAUNCH;
     if (marks) mark(g_ev_stop);
     cfg.gridDim = dim3(static_cast<unsigned>(cgrid));
     cfg.blockDim = dim3(COMBINE_THREADS);
@@ -602,6 +645,7 @@ int launch_decode(DeviceState* st, const void* q, const void* kc, const void* vc
     p.g = g;
     p.n_hb = n_hb;
     p.P = P;
+    p.self_in_cache = g_self_in_cache;
     p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
     p.rope = rope_spec(theta);
     p.scale_log2 *= rope_mscale() * rope_mscale();   // YaRN temperature (1 without scaling)
@@ -668,6 +712,7 @@ int launch_decode_fixed_scratch(DeviceState* st, const void* q, const void* kc, 
     p.g = g;
     p.n_hb = n_hb;
     p.P = P;
+    p.self_in_cache = g_self_in_cache;
     p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
     p.rope = rope_spec(theta);
     p.scale_log2 *= rope_mscale() * rope_mscale();   // YaRN temperature (1 without scaling)
@@ -800,6 +845,35 @@ int gqa_qkv_rope(const void* x, const void* w_qkv, const void* b_qkv, void* qr, 
     if (!st) return rc;
     return d == 64 ? launch_qkv<64>(st, x, w_qkv, b_qkv, qr, kr, k, v, B, L, d_model, h_q, h_kv, theta)
                    : launch_qkv<128>(st, x, w_qkv, b_qkv, qr, kr, k, v, B, L, d_model, h_q, h_kv, theta);
+}
+
+int gqa_qkv_append(const void* x, const void* w_qkv, const void* b_qkv, const int* seqlens, void* q, void* kpages,
+                   void* vpages, const int* block_table, int B, int d_model, int h_q, int h_kv, int d, int page_size,
+                   int num_pages, int max_pages_per_seq) {
+    if (B < 0 || d_model <= 0 || d_model % 8 != 0 || page_size <= 0 || num_pages <= 0 || max_pages_per_seq <= 0)
+        return GQA_ERR_DIMS;
+    if (static_cast<long long>(num_pages) * page_size > (1LL << 40)) return GQA_ERR_DIMS;
+    if (static_cast<long long>(B) * max_pages_per_seq > 0x7fffffffLL) return GQA_ERR_DIMS;
+    int rc = check_common(h_q, h_kv, d, 1.0f);
+    if (rc != GQA_OK) return rc;
+    if (B == 0) return GQA_OK;
+    if (!x || !w_qkv || !seqlens || !q || !kpages || !vpages || !block_table) return GQA_ERR_NULL;
+    if (!aligned16(x) || !aligned16(w_qkv) || !aligned16(q) || !aligned16(kpages) || !aligned16(vpages) ||
+        (b_qkv && !aligned16(b_qkv)))
+        return GQA_ERR_ALIGN;
+    if (static_cast<long long>(h_q + 2 * h_kv) * d > 0x7fffffffLL) return GQA_ERR_DIMS;
+    DeviceState* st = device_state(&rc);
+    if (!st) return rc;
+    return d == 64 ? launch_append<64>(st, x, w_qkv, b_qkv, seqlens, q, kpages, vpages, block_table, B, d_model, h_q,
+                                       h_kv, page_size, num_pages, max_pages_per_seq)
+                   : launch_append<128>(st, x, w_qkv, b_qkv, seqlens, q, kpages, vpages, block_table, B, d_model,
+                                        h_q, h_kv, page_size, num_pages, max_pages_per_seq);
+}
+
+int gqa_set_decode_self_in_cache(int on) {
+    if (on != 0 && on != 1) return GQA_ERR_DIMS;
+    g_self_in_cache = on;
+    return GQA_OK;
 }
 
 int gqa_out_proj(const void* attn, const void* w_o, const void* residual, void* out, int T, int d_in, int d_model) {

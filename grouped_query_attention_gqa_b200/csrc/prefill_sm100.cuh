@@ -25,12 +25,13 @@
 //   warps 0-3  softmax for query tile 0   (thread = query row = TMEM lane)
 //   warps 4-7  softmax for query tile 1
 //   warp  8    TMA producer of K', V tiles (2-stage rings)
-//   warp  9    tcgen05 MMA issuer (one thread); also owns the TMEM allocation
+//   warp  9    tcgen05 MMA issuer (the whole warp, converged; one elected lane issues each MMA);
+//              also owns the TMEM allocation
 //   warp 10    TMA producer of the Q' tiles (one buffer per query tile)
 //   warp 11    idle
 // Each SM sub-partition hosts three warps, which caps a uniform budget at 168
-// registers; the third warpgroup hands 88 of its registers per thread to the
-// two softmax warpgroups (setmaxnreg: 208 / 208 / 80), which then hold a full
+// registers; the third warpgroup hands 80 of its registers per thread to the
+// two softmax warpgroups (setmaxnreg: 208 / 208 / 88), which then hold a full
 // 128-column score row in registers.
 // Tensor memory (512 columns): S0 [0,128) S1 [128,256) O0 [256,256+d) O1 [.., +d);
 // P_k (bf16, two per column) overwrites the first 64 columns of S_k.
@@ -57,18 +58,20 @@ constexpr int WARP_TMA = 8;     // K'/V producer
 constexpr int WARP_MMA = 9;
 constexpr int WARP_QLOAD = 10;  // Q' producer
 // Register split.  setmaxnreg.inc waits until the registers exist in the block's own
-// allocation (threads x launch registers), so the shares must not add up to more than that;
+// allocation (threads x launch registers), so the shares must not add up to more than that
+// (here they add up to it exactly: 256 x 208 + 128 x 88 = 384 x 168);
 // the host refuses to launch if ptxas gave the kernel any other count than LAUNCH_REGS.
 constexpr int LAUNCH_REGS = 168;
 constexpr int SOFTMAX_REGS = 208;
-constexpr int OTHER_REGS = 80;
+constexpr int OTHER_REGS = 88;
 static_assert(256 * SOFTMAX_REGS + 128 * OTHER_REGS <= NUM_THREADS * LAUNCH_REGS, "register split");
 constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t P_COL = 0;    // P_k (128 bf16 per row, two per column) fills columns 0..63 of S_k
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: O is rescaled only when the max grows by > 2^8
 // Of every 8 consecutive pairs of exponentials of a row (off the diagonal tile), this many run on
 // the FMA pipe (exp2_poly_x2) and the rest on the ex2 unit.
 #ifndef GQA_EXP_POLY_OF_8
-#define GQA_EXP_POLY_OF_8 1
+#define GQA_EXP_POLY_OF_8 2
 #endif
 #ifndef GQA_PREP_POS
 #define GQA_PREP_POS 8
@@ -218,12 +221,12 @@ __global__ void __launch_bounds__(PREP_THREADS, GQA_PREP_MIN_CTAS) prep_kernel(c
     }
 }
 
-// P = 2^(s * scale_log2 - m) for one row of 128 scores, stored as bf16 pairs into the first 64
-// columns of the S region (chunk c overwrites S columns 16c.., already in registers); returns the
-// row sum of the fp32 values.  POLY: part of the exponentials on the FMA pipe (never on a tile
+// P = 2^(s * scale_log2 - m) for one row of 128 scores, stored as bf16 pairs from TMEM column t_p
+// (the first half of the S region: chunk c overwrites S columns 16c.., already in registers); returns
+// the row sum of the fp32 values.  POLY: part of the exponentials on the FMA pipe (never on a tile
 // with masked entries, whose weights must be exactly 0).
 template <bool POLY>
-__device__ __forceinline__ float row_exp_store(const uint32_t (&sr)[4][32], float sl2, float neg_m, uint32_t t_s) {
+__device__ __forceinline__ float row_exp_store(const uint32_t (&sr)[4][32], float sl2, float neg_m, uint32_t t_p) {
     const uint64_t scale2 = f2_pack(sl2, sl2), shift2 = f2_pack(neg_m, neg_m);
     uint64_t acc[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
 #pragma unroll
@@ -244,7 +247,7 @@ __device__ __forceinline__ float row_exp_store(const uint32_t (&sr)[4][32], floa
             acc[(e >> 1) & 1] = f2_add(acc[(e >> 1) & 1], f2_pack(p0, p1));
             pk[e >> 1] = pack_bf16x2(p0, p1);
         }
-        tmem_st16(t_s + 16 * c, pk);
+        tmem_st16(t_p + 16 * c, pk);
     }
     float a0, a1, b0, b1;
     f2_unpack(acc[0], a0, a1);
@@ -353,6 +356,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int r = (warp & 3) * 32 + lane;   // query row in the tile == TMEM lane
         const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
         const uint32_t t_s = tmem + lane_base + static_cast<uint32_t>(k * 128);
+        const uint32_t t_p = t_s + P_COL;   // P_k: bf16 pairs over the first half of S_k
         const uint32_t t_o = tmem + lane_base + static_cast<uint32_t>(256 + k * D);
         const float sl2 = p.scale_log2;
         uint32_t s_seen = 0;   // S_k results consumed (s_full phases)
@@ -412,8 +416,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     tmem_wait_st();
                 }
                 const float neg_m = -m_run;
-                if (diag) l_run += row_exp_store<false>(sr, sl2, neg_m, t_s);
-                else l_run += row_exp_store<true>(sr, sl2, neg_m, t_s);
+                if (diag) l_run += row_exp_store<false>(sr, sl2, neg_m, t_p);
+                else l_run += row_exp_store<true>(sr, sl2, neg_m, t_p);
                 tmem_wait_st();
                 tc_fence_before();
                 mbar_arrive(&sh.p_full[k]);
@@ -534,30 +538,37 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
     } else if (warp == WARP_MMA) {
         // ================================================================ MMA issuer
-        if (lane == 0) {
+        // The whole warp runs the loop, converged, on warp-uniform state; one elected lane issues each
+        // tcgen05 instruction.  Descriptors are formed once and advanced by constant offsets.
+        {
             constexpr uint32_t IDESC_S = idesc_bf16_f32(BM, BN, false);
             constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, D, true);
-            const uint32_t q_addr0 = smem_u32(smem + Lay::Q0);
-            const uint32_t k_addr0 = smem_u32(smem + Lay::K0);
-            const uint32_t v_addr0 = smem_u32(smem + Lay::V0);
+            const uint32_t tm = tmem;   // read from shared memory: the same in every lane
+            // The descriptors' low words (start address and leading offset); the high words are constants.
+            const uint32_t q_lo = static_cast<uint32_t>(sw128_desc(smem_u32(smem + Lay::Q0), 16, 1024));
+            const uint32_t k_lo = static_cast<uint32_t>(sw128_desc(smem_u32(smem + Lay::K0), 16, 1024));
+            const uint32_t v_lo = static_cast<uint32_t>(sw128_desc(smem_u32(smem + Lay::V0), Lay::SUB, 1024));
+            constexpr uint64_t DESC_HI = sw128_desc(0, 0, 1024) & 0xFFFFFFFF00000000ull;
+            constexpr uint32_t TILE16 = Lay::TILE >> 4;   // one tile in descriptor address units
             // S_k = Q_k K_j^T : M=128 (query rows), N=128 (key rows), K=D in steps of 16.
             auto issue_s = [&](int k, int ks) {
-                const uint32_t qa = q_addr0 + k * Lay::TILE;
-                const uint32_t ka = k_addr0 + ks * Lay::TILE;
+                const uint32_t qa = q_lo + static_cast<uint32_t>(k) * TILE16;
+                const uint32_t ka = k_lo + static_cast<uint32_t>(ks) * TILE16;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = static_cast<uint32_t>((kk >> 2) * Lay::SUB + (kk & 3) * 32);
-                    umma_ss(tmem + static_cast<uint32_t>(k * 128), sw128_desc(qa + off, 16, 1024),
-                            sw128_desc(ka + off, 16, 1024), IDESC_S, kk > 0 ? 1u : 0u);
+                    const uint32_t off = static_cast<uint32_t>(((kk >> 2) * Lay::SUB + (kk & 3) * 32) >> 4);
+                    umma_ss_warp(tm + static_cast<uint32_t>(k * 128), DESC_HI | (qa + off), DESC_HI | (ka + off),
+                                 IDESC_S, kk > 0 ? 1u : 0u);
                 }
             };
             // O_k += P_k V_j : M=128, N=D (V is MN-major: d contiguous), K=128 key rows in steps of 16.
             auto issue_pv = [&](int k, int vs, bool acc) {
-                const uint32_t va = v_addr0 + vs * Lay::TILE;
+                const uint32_t va = v_lo + static_cast<uint32_t>(vs) * TILE16;
 #pragma unroll
                 for (int kk = 0; kk < BN / 16; ++kk) {
-                    umma_ts(tmem + static_cast<uint32_t>(256 + k * D), tmem + static_cast<uint32_t>(k * 128 + kk * 8),
-                            sw128_desc(va + kk * 16 * 128, Lay::SUB, 1024), IDESC_PV, (acc || kk > 0) ? 1u : 0u);
+                    umma_ts_warp(tm + static_cast<uint32_t>(256 + k * D), tm + static_cast<uint32_t>(k * 128 + P_COL + kk * 8),
+                                 DESC_HI | (va + static_cast<uint32_t>(kk * 16 * 128 >> 4)), IDESC_PV,
+                                 (acc || kk > 0) ? 1u : 0u);
                 }
             };
             uint32_t kv = 0;               // K/V tiles consumed (ring position)
@@ -565,64 +576,63 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             uint32_t pn[2] = {0u, 0u};     // p_full phases consumed per tile
             bool ok = true;
             for (int it = 0; ok; ++it) {
-                const int w = work_item(p, it, cta, G);
+                const int w = __shfl_sync(0xffffffffu, work_item(p, it, cta, G), 0);
                 if (w >= p.total_work) break;
                 const PairWork pw = pair_work(p, w);
                 const int n[2] = {pw.n0, pw.n1};
                 const int nmax = n[0] > n[1] ? n[0] : n[1];
                 // S_k of the first key tile as soon as query tile k is in shared memory.
                 const int ks0 = kv % KSTAGES;
-                ok = mbar_wait(&sh.k_full[ks0], (kv / KSTAGES) & 1, p.err, abort);
+                ok = mbar_wait_warp(&sh.k_full[ks0], (kv / KSTAGES) & 1, p.err, abort);
                 for (int k = 0; k < 2 && ok; ++k) {
                     if (n[k] == 0) continue;
-                    ok = mbar_wait(&sh.q_full[k], qn[k] & 1, p.err, abort);
+                    ok = mbar_wait_warp(&sh.q_full[k], qn[k] & 1, p.err, abort);
                     if (!ok) break;
                     ++qn[k];
                     tc_fence_after();
                     issue_s(k, ks0);
-                    umma_commit(&sh.s_full[k]);
-                    if (n[k] == 1) umma_commit(&sh.q_empty[k]);   // that was the last S on buffer k
+                    umma_commit_warp(&sh.s_full[k]);
+                    if (n[k] == 1) umma_commit_warp(&sh.q_empty[k]);   // that was the last S on buffer k
                 }
                 if (!ok) break;
-                umma_commit(&sh.k_empty[ks0]);
+                umma_commit_warp(&sh.k_empty[ks0]);
                 for (int j = 0; j < nmax && ok; ++j) {
                     const uint32_t vi = kv + j;
                     const int vs = vi % VSTAGES;
-                    ok = mbar_wait(&sh.v_full[vs], (vi / VSTAGES) & 1, p.err, abort);
+                    ok = mbar_wait_warp(&sh.v_full[vs], (vi / VSTAGES) & 1, p.err, abort);
                     if (!ok) break;
                     bool k_next = false;
                     const uint32_t ki = kv + j + 1;
                     for (int k = 0; k < 2 && ok; ++k) {
                         if (j >= n[k]) continue;
-                        ok = mbar_wait(&sh.p_full[k], pn[k] & 1, p.err, abort);
+                        ok = mbar_wait_warp(&sh.p_full[k], pn[k] & 1, p.err, abort);
                         if (!ok) break;
                         ++pn[k];
                         tc_fence_after();
                         issue_pv(k, vs, j > 0);
-                        umma_commit(&sh.o_full[k]);
+                        umma_commit_warp(&sh.o_full[k]);
                         if (j + 1 < n[k]) {
                             if (!k_next) {
-                                ok = mbar_wait(&sh.k_full[ki % KSTAGES], (ki / KSTAGES) & 1, p.err, abort);
+                                ok = mbar_wait_warp(&sh.k_full[ki % KSTAGES], (ki / KSTAGES) & 1, p.err, abort);
                                 if (!ok) break;
                                 tc_fence_after();
                                 k_next = true;
                             }
                             issue_s(k, ki % KSTAGES);
-                            umma_commit(&sh.s_full[k]);
-                            if (j + 2 == n[k]) umma_commit(&sh.q_empty[k]);
+                            umma_commit_warp(&sh.s_full[k]);
+                            if (j + 2 == n[k]) umma_commit_warp(&sh.q_empty[k]);
                         }
                     }
-                    umma_commit(&sh.v_empty[vs]);
-                    if (k_next) umma_commit(&sh.k_empty[ki % KSTAGES]);
+                    umma_commit_warp(&sh.v_empty[vs]);
+                    if (k_next) umma_commit_warp(&sh.k_empty[ki % KSTAGES]);
                 }
                 kv += nmax;
             }
             // Every MMA must have finished before the tensor memory is released.
-            umma_commit(&sh.mma_done);
-            mbar_wait(&sh.mma_done, 0, p.err, nullptr);
+            umma_commit_warp(&sh.mma_done);
+            mbar_wait_warp(&sh.mma_done, 0, p.err, nullptr);
         }
     }
-
     tc_fence_before();
     __syncthreads();
     if (warp == WARP_MMA) {

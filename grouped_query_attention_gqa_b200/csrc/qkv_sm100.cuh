@@ -65,6 +65,12 @@ struct Params {
     __nv_bfloat16* v;
     const __nv_bfloat16* resid;  // output projection: residual [T, N] or nullptr
     __nv_bfloat16* out;          // output projection: out [T, N] (may be resid itself)
+    // Decode-step append (kAppend): token t is the new token of sequence t, at position seqlens[t]; q goes
+    // to qr [T, h_q, d], its K and V rows to the page slot of that position in k / v, the key and value
+    // pages [num_pages, page_size, h_kv, d], through the block table bt [T, max_pages].
+    const int* seqlens;
+    const int* bt;
+    int page_size, max_pages, num_pages;
     int T, L, N, h_q, h_kv;
     int n_ntiles, n_tiles, kblocks;
     // Work units: tiles 0 .. n_main-1 whole (BN columns); each later tile split into tail_split units of
@@ -242,11 +248,39 @@ __device__ __forceinline__ void store_resid(const Params& p, float (&y)[W], int 
     store_rows<W>(stage, valid ? p.out + at : nullptr, y, lane);
 }
 
-enum Epilogue { kQKV = 0, kResidual = 1 };
+// The decode-step append's epilogue: one head of one token row per lane, + bias, stored un-rotated (the
+// decode rotates q and every cached key at its position): a query head to its q row, a key or value head
+// to the token's page slot (kv_row: the slot's row of h_kv heads in the key or value pages, nullptr when
+// the row is past the end or its table entry is invalid).
+template <int D>
+__device__ __forceinline__ void store_append(const Params& p, float (&y)[D], int n0, int t, bool valid,
+                                             __nv_bfloat16* k_row, __nv_bfloat16* v_row, uint8_t* stage, int lane) {
+    if (p.bias) {
+        const uint4* bb = reinterpret_cast<const uint4*>(p.bias + n0);
+#pragma unroll
+        for (int c = 0; c < D / 8; ++c) {
+            const uint4 w = bb[c];
+            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                y[8 * c + 2 * e] += bf16lo_to_f32(ws[e]);
+                y[8 * c + 2 * e + 1] += bf16hi_to_f32(ws[e]);
+            }
+        }
+    }
+    const int head = n0 / D;
+    __nv_bfloat16* dst;
+    if (head < p.h_q) dst = valid ? p.qr + (static_cast<int64_t>(t) * p.h_q + head) * D : nullptr;
+    else if (head < p.h_q + p.h_kv) dst = k_row ? k_row + static_cast<int64_t>(head - p.h_q) * D : nullptr;
+    else dst = v_row ? v_row + static_cast<int64_t>(head - p.h_q - p.h_kv) * D : nullptr;
+    store_rows<D>(stage, dst, y, lane);
+}
+
+enum Epilogue { kQKV = 0, kResidual = 1, kAppend = 2 };
 
 // ---------------------------------------------------------------------------------------------
-// The persistent GEMM: Y[T, N] = X[T, K] W[N, K]^T with the epilogue EPI.  For kQKV, D is the head size
-// (tiles are processed head by head); for kResidual, D = 128 (tiles are processed 128 columns at a time).
+// The persistent GEMM: Y[T, N] = X[T, K] W[N, K]^T with the epilogue EPI.  For kQKV and kAppend, D is the
+// head size (tiles are processed head by head); for kResidual, D = 128 (128 columns at a time).
 template <int D, int EPI, int BN_>
 __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtensorMap& tm_w, const CUtensorMap& tm_wt,
                                           const Params& p) {
@@ -410,6 +444,20 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtenso
             const int t = un.mt * BM + r;
             const bool valid = t < p.T;
             const int b = valid ? t / p.L : 0, pos = valid ? t % p.L : 0;
+            // kAppend: this row's page slot (rows of all h_kv heads) in the key and value pages
+            __nv_bfloat16 *k_row = nullptr, *v_row = nullptr;
+            if (EPI == kAppend && valid) {
+                const int at = __ldg(p.seqlens + t);
+                const int pi = at >= 0 ? at / p.page_size : -1;
+                const int page = (pi >= 0 && pi < p.max_pages) ? __ldg(p.bt + static_cast<int64_t>(t) * p.max_pages + pi) : -1;
+                if (page >= 0 && page < p.num_pages) {
+                    const int64_t slot = static_cast<int64_t>(page) * p.page_size + (at - pi * p.page_size);
+                    k_row = p.k + slot * p.h_kv * D;
+                    v_row = p.v + slot * p.h_kv * D;
+                } else if (un.n0 == 0) {
+                    atomicOr(p.err, kErrBadPage);   // once per row: nothing of this token is cached
+                }
+            }
             if (EPI == kResidual && un.width == TAIL_BN) {
                 // A tail unit (output projection only): its 64 columns in one pass.
                 if (un.n0 < p.N) {
@@ -433,6 +481,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtenso
                                   *reinterpret_cast<uint32_t(*)[32]>(acc + 32 * c));
                     tmem_wait_ld();
                     if (EPI == kQKV) store_head<D>(p, acc, n0, b, pos, valid, stage, lane);
+                    else if (EPI == kAppend) store_append<D>(p, acc, n0, t, valid, k_row, v_row, stage, lane);
                     else store_resid<128>(p, *reinterpret_cast<float(*)[128]>(acc), n0, t, valid, stage, lane);
                 }
             }
@@ -455,6 +504,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     qkv_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
                const __grid_constant__ CUtensorMap tm_wt, const Params p) {
     gemm_body<D, kQKV, BN>(tm_x, tm_w, tm_wt, p);
+}
+
+// One decode step's projection and cache append (page "Qwen2 architecture introduction", §4.1.3 steps 1-2
+// and closing paragraph: the current token's K and V are appended to the cache each step): x [T, d_model]
+// holds the new token of T sequences; q [T, h_q, D] and the page slots of positions seqlens[t] get the
+// un-rotated heads.
+template <int D, int BN>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    append_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
+                  const __grid_constant__ CUtensorMap tm_wt, const Params p) {
+    gemm_body<D, kAppend, BN>(tm_x, tm_w, tm_wt, p);
 }
 
 // Output projection + residual (page "Qwen2 architecture introduction", §4.1.3 steps 5-6):

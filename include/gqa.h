@@ -171,6 +171,42 @@ GQA_API int gqa_qkv_rope(const void* x, const void* w_qkv, const void* b_qkv, vo
                          int B, int L, int d_model, int h_q, int h_kv, int d, float theta);
 
 /*
+ * gqa_qkv_append -- one decode step's projection with its cache append (page "Qwen2 architecture
+ * introduction", aicoding.csdn.net, §4.1.3 steps 1-2 and closing paragraph: each decode step projects the
+ * new token and appends its K and V to the cache of the h_kv groups; page "从 Qwen 1 到 Qwen 2", nxmr.cn,
+ * §2.4: that cache kept in pages, as gqa_decode_paged reads it).
+ *   x            [B, d_model]  the new token of each of B sequences (hidden states after RMSNorm), bf16
+ *   w_qkv, b_qkv as for gqa_qkv_rope (b_qkv may be NULL)
+ *   seqlens      [B] int32, DEVICE memory: each sequence's cache length before the append, i.e. the
+ *                position p_b of its new token
+ *   q            [B, h_q, d]   out: the new tokens' queries, un-rotated (the decode entry points rotate the
+ *                query at its position)
+ *   kpages, vpages [num_pages, page_size, h_kv, d]  the paged cache of gqa_decode_paged: the token's K
+ *                (un-rotated, like every cache row) and V are written to slot p_b % page_size of page
+ *                block_table[b][p_b / page_size]; nothing else in the pages is touched
+ *   block_table  [B, max_pages_per_seq] int32, DEVICE memory
+ * Each written element is the fp32 accumulation (plus the bias) rounded once to bf16.  A decode loop is
+ * then: gqa_qkv_append, then gqa_decode_paged with seqlens[b] + 1 and gqa_set_decode_self_in_cache(1) (the
+ * new token attends to itself and to every earlier position), then grow seqlens.  A position outside the
+ * table (p_b < 0, or p_b / page_size >= max_pages_per_seq) or a table entry outside [0, num_pages) is not
+ * an API error (both live on the device): that token's K and V are not written and GQA_DEVERR_PAGE is
+ * raised; its q is still written.  Sizes as for gqa_qkv_rope and gqa_decode_paged; B == 0 is a no-op.
+ */
+GQA_API int gqa_qkv_append(const void* x, const void* w_qkv, const void* b_qkv, const int* seqlens, void* q,
+                           void* kpages, void* vpages, const int* block_table, int B, int d_model, int h_q,
+                           int h_kv, int d, int page_size, int num_pages, int max_pages_per_seq);
+
+/*
+ * gqa_set_decode_self_in_cache -- where the query of every later gqa_decode, gqa_decode_paged and
+ * gqa_decode_noalloc call sits.  0 (the default): at position seqlens[b], attending to the seqlens[b]
+ * cached rows before it, which do not include the query's own row.  1: the cache already holds the query's
+ * own K and V as its last row (appended by gqa_qkv_append, the order of page "Qwen2 architecture
+ * introduction", §4.1.3 closing paragraph), so the query sits at position seqlens[b] - 1 and attends to all
+ * seqlens[b] rows, itself included.  Process-global, like the stream.  Returns GQA_ERR_DIMS for other values.
+ */
+GQA_API int gqa_set_decode_self_in_cache(int on);
+
+/*
  * gqa_prefill_rotated -- the causal attention of gqa_prefill on inputs that are already rotated (page
  * "Qwen2 architecture introduction", §4.1.3 steps 4-5): qr [B, h_q, L, d] and kr [B, h_kv, L, d]
  * head-major as gqa_qkv_rope writes them, v [B, L, h_kv, d], out [B, L, h_q, d].  No RoPE and no

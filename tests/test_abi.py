@@ -32,7 +32,8 @@ def codes():
 def test_header_declares_the_entry_points():
     names = set(declared())
     for n in ["gqa_prefill", "gqa_decode", "gqa_decode_paged", "gqa_qkv_rope", "gqa_prefill_rotated",
-              "gqa_out_proj", "gqa_set_stream", "gqa_last_error", "gqa_release",
+              "gqa_out_proj", "gqa_qkv_append", "gqa_set_decode_self_in_cache", "gqa_set_stream", "gqa_last_error",
+              "gqa_release",
               "gqa_strerror", "gqa_abi_version", "gqa_set_timing_events"]:
         assert n in names
 
@@ -169,3 +170,36 @@ def test_set_rope_scaling_validation(lib, factor, orig, code):
 
 def test_set_stream_accepts_null(lib):
     assert lib.gqa_set_stream(None) == 0
+
+
+def append_args(x=P16, w=P16, b=None, s=P16, q=P16, kp=P16, vp=P16, bt=P16, B=2, dm=256, h_q=28, h_kv=4, d=128,
+                page=16, npages=8, maxp=4):
+    return (x, w, b, s, q, kp, vp, bt, B, dm, h_q, h_kv, d, page, npages, maxp)
+
+
+@pytest.mark.parametrize("args,code", [
+    (append_args(B=-1), "GQA_ERR_DIMS"),
+    (append_args(dm=0), "GQA_ERR_DIMS"),
+    (append_args(dm=100), "GQA_ERR_DIMS"),          # not a multiple of 8
+    (append_args(page=0), "GQA_ERR_DIMS"),
+    (append_args(npages=0), "GQA_ERR_DIMS"),
+    (append_args(maxp=0), "GQA_ERR_DIMS"),
+    (append_args(npages=1 << 30, page=1 << 12), "GQA_ERR_DIMS"),      # storage rows beyond 2^40
+    (append_args(h_kv=3), "GQA_ERR_DIMS"),
+    (append_args(d=96), "GQA_ERR_HEAD_DIM"),
+    (append_args(x=None), "GQA_ERR_NULL"),
+    (append_args(s=None), "GQA_ERR_NULL"),
+    (append_args(bt=None), "GQA_ERR_NULL"),
+    (append_args(kp=None), "GQA_ERR_NULL"),
+    (append_args(b=ctypes.c_void_p(264)), "GQA_ERR_ALIGN"),
+    (append_args(vp=ctypes.c_void_p(8)), "GQA_ERR_ALIGN"),
+    (append_args(x=None, w=None, s=None, q=None, kp=None, vp=None, bt=None, B=0), "GQA_OK"),
+])
+def test_qkv_append_validation(lib, args, code):
+    assert lib.gqa_qkv_append(*args) == codes()[code]
+
+
+@pytest.mark.parametrize("on,code", [(0, "GQA_OK"), (1, "GQA_OK"), (2, "GQA_ERR_DIMS"), (-1, "GQA_ERR_DIMS")])
+def test_set_decode_self_in_cache_validation(lib, on, code):
+    assert lib.gqa_set_decode_self_in_cache(on) == codes()[code]
+    lib.gqa_set_decode_self_in_cache(0)
