@@ -331,16 +331,17 @@ def release() -> None:
 def prefill_schedule(B: int, L: int, h_q: int, h_kv: int, grid: int):
     """The attention work schedule gqa_prefill uses for this shape over `grid` CTAs (host only).
 
-    Returns (lists, snake): lists[c] is CTA c's item list in order; snake is True where the library keeps
-    its round-robin order instead (the lists are then those of the packing it compared against).
+    Returns (lists, grouped): lists[c] is CTA c's item list in order; grouped is True where the items are
+    dealt plane group by plane group for L2 reuse (many items per CTA), False where they are packed by
+    best fit for balance.
     """
     lib = load()
-    snake = ctypes.c_int(0)
-    n = lib.gqa_prefill_schedule(B, L, h_q, h_kv, grid, None, None, 0, ctypes.byref(snake))
+    grouped = ctypes.c_int(0)
+    n = lib.gqa_prefill_schedule(B, L, h_q, h_kv, grid, None, None, 0, ctypes.byref(grouped))
     if n < 0:
         raise GQAError(n, "gqa_prefill_schedule")
     g = min(grid, n)
     starts = (ctypes.c_int * (g + 1))()
     items = (ctypes.c_int * max(n, 1))()
-    lib.gqa_prefill_schedule(B, L, h_q, h_kv, grid, starts, items, n, ctypes.byref(snake))
-    return [list(items[starts[c]:starts[c + 1]]) for c in range(g)], bool(snake.value)
+    lib.gqa_prefill_schedule(B, L, h_q, h_kv, grid, starts, items, n, ctypes.byref(grouped))
+    return [list(items[starts[c]:starts[c + 1]]) for c in range(g)], bool(grouped.value)

@@ -40,6 +40,9 @@ using namespace ptx;
 #ifndef GQA_DECODE_STAGES
 #define GQA_DECODE_STAGES 2
 #endif
+#ifndef GQA_PAGED_TRACK
+#define GQA_PAGED_TRACK 1
+#endif
 #ifndef GQA_DECODE_CTAS_PER_SM
 #define GQA_DECODE_CTAS_PER_SM 3
 #endif
@@ -243,6 +246,14 @@ __global__ void __launch_bounds__(WARPS * 32, CTAS_PER_SM) split_kernel(const Pa
     const uint64_t stream_policy = l2_evict_first_policy();
     BlockCursor iss;
     iss.init(p.off, p.B, start, end);
+#if GQA_PAGED_TRACK
+    // Paged, pages of >= 16 rows: the producer's current piece (sequence pg_b), the page index and offset
+    // of its block's first row, and the table entries of that page and the next (-1: past the table).
+    int pg_b = -1, pg_idx = 0, pg_rem = 0, pg_cur = -1, pg_next = -1;
+    auto table_entry = [&](int b, int pi) {
+        return pi < p.max_pages ? __ldg(p.bt + static_cast<int64_t>(b) * p.max_pages + pi) : -1;
+    };
+#endif
     auto issue = [&](int stage) {
         const int nvalid = static_cast<int>(iss.seg_end - iss.r < ROWS ? iss.seg_end - iss.r : ROWS);
         uint64_t* bar = &bars[warp][stage];
@@ -253,6 +264,40 @@ __global__ void __launch_bounds__(WARPS * 32, CTAS_PER_SM) split_kernel(const Pa
         // row stays zero and the device error word gets kErrBadPage.
         bool load = i < nvalid;
         int64_t srow = iss.r + i;
+#if GQA_PAGED_TRACK
+        if (PAGED && p.page_size >= ROWS) {
+            // Pages of at least 16 rows: a block spans at most two of them.  The block's page and the next
+            // one are tracked from block to block (the next table entry read one page ahead), so a block
+            // costs no division and no table read on its path.
+            const int ps = p.page_size;
+            if (iss.b != pg_b) {   // a new piece: locate its first block once (warp-uniform)
+                pg_b = iss.b;
+                const int j0 = static_cast<int>(iss.r - p.off[iss.b]);   // position in the sequence (< 2^31)
+                pg_idx = j0 / ps;
+                pg_rem = j0 - pg_idx * ps;
+                pg_cur = table_entry(pg_b, pg_idx);
+                pg_next = table_entry(pg_b, pg_idx + 1);
+            } else {
+                pg_rem += ROWS;
+                if (pg_rem >= ps) {
+                    pg_rem -= ps;
+                    ++pg_idx;
+                    pg_cur = pg_next;
+                    pg_next = table_entry(pg_b, pg_idx + 1);
+                }
+            }
+            const int t = pg_rem + i;
+            const int page = t < ps ? pg_cur : pg_next;
+            if (load) {
+                if (page < 0 || page >= p.num_pages) {
+                    load = false;
+                    atomicOr(p.err, kErrBadPage);
+                } else {
+                    srow = static_cast<int64_t>(page) * ps + (t < ps ? t : t - ps);
+                }
+            }
+        } else
+#endif
         if (PAGED && load) {
             const int j = static_cast<int>(srow - p.off[iss.b]);   // position in the sequence (< 2^31)
             const int pi = j / p.page_size;

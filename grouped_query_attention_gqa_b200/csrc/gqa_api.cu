@@ -49,7 +49,7 @@ struct DeviceState {
     CUtensorMap maps[4];
     // The attention kernel's work schedule for the last (B, L, h_q, h_kv, grid): per-CTA item lists (CSR).
     int sched_key[5] = {0, 0, 0, 0, 0};
-    bool sched_valid = false, sched_snake = true;
+    bool sched_valid = false;
     void* sched = nullptr;
     size_t sched_bytes = 0;
     // QKV projection: the cos / sin table of the last (L, d, theta), and the last pair of tensor maps.
@@ -225,16 +225,40 @@ int encode_prefill_maps(CUtensorMap* maps, const void* qr, const void* kr, const
 #define GQA_SCHED_ITEM_COST 4
 #endif
 
+// KV planes dealt together when there are many items per CTA, sized for d = 128 whatever d is (the
+// schedule is planned without d).  Where the K' and V of all planes fit in well under half of the 126 MB L2
+// (48 MB), all of them (no grouping: measured, grouping then only loses the round-robin's order, 3 % at
+// B=2, L=8192); otherwise as many as keep 16 MB of K' and V, at least one.  Measured against all planes at
+// once on B=4, L=8192 with 64/8 heads (32 planes of 4 MB): groups of 16 MB 8 % fewer cycles per launch,
+// of 32 or 64 MB 1-3 %; at L=32768 (4 planes of 16.8 MB, one at a time) 1 %.
+#ifndef GQA_GROUP_KV_BYTES
+#define GQA_GROUP_KV_BYTES (16ll << 20)
+#endif
+#ifndef GQA_GROUP_ALL_KV_BYTES
+#define GQA_GROUP_ALL_KV_BYTES (48ll << 20)
+#endif
+int attention_group_planes(int B, int L, int h_kv) {
+    const long long per_plane = 2LL * L * 128 * 2;   // K' and V of one (b, u) plane at d = 128
+    const long long planes = static_cast<long long>(B) * h_kv;
+    if (planes * per_plane <= GQA_GROUP_ALL_KV_BYTES) return static_cast<int>(planes);
+    long long g = GQA_GROUP_KV_BYTES / (per_plane > 0 ? per_plane : 1);
+    if (g < 1) g = 1;
+    if (g > planes) g = planes;
+    return static_cast<int>(g);
+}
+
 // The attention kernel's work schedule: which items (pairs of query tiles, numbered as in the kernel's
 // pair_work) each persistent CTA processes, in order.  Item w costs the key tiles of its two query tiles
-// plus a fixed overhead; the items are dealt heaviest first, each to the fullest CTA that still has room
-// below a capacity (best fit decreasing), the capacity raised from its lower bound -- the mean load or the
-// largest item -- until everything fits.  With 3 items per CTA (Qwen2-7B, L=4096: 448 items over 148 CTAs)
-// the kernel's own round-robin (snake) order leaves the busiest CTA with 9 % more work than the average;
-// this reaches the average.  With many items per CTA the snake order is already within 2 % of it and is
-// kept (*use_snake).  Built on the host once per shape and kept on the device (CSR: starts[grid + 1], items).
+// plus a fixed overhead.  With few items per CTA (Qwen2-7B, L=4096: 448 items over 148 CTAs) the balance
+// is what matters: the items are dealt heaviest first, each to the fullest CTA that still has room below
+// a capacity (best fit decreasing), the capacity raised from its lower bound -- the mean load or the
+// largest item -- until everything fits; a round-robin (snake) order would leave the busiest CTA with 9 %
+// more work than the average.  With many items per CTA (where that snake order is already within 2 % of
+// the packing) any dealing balances: the snake order itself where every plane's K' and V fit L2, else the
+// items are dealt for L2 reuse, plane group by plane group (*grouped).  Built on the host once per shape and
+// kept on the device (CSR: starts[grid + 1], items).
 // Pure host computation of that schedule for B batch rows, L positions, h_q / h_kv heads and `grid` CTAs:
-// fills csr (starts[grid + 1], then the items) and returns true if the snake order is kept instead.
+// fills csr (starts[grid + 1], then the items) and returns true for the plane-grouped dealing.
 bool plan_attention_schedule(int B, int L, int h_q, int h_kv, int grid, std::vector<int>& csr) {
     constexpr int BM = gqa::prefill::BM;
     const int n_qtiles = (L + BM - 1) / BM, g = h_q / h_kv;
@@ -282,6 +306,41 @@ bool plan_attention_schedule(int B, int L, int h_q, int h_kv, int grid, std::vec
         if (fits) break;
         cap += std::max(1LL, cap / 256);
     }
+    const bool many = 100 * snake_max <= 102 * cap;
+    const int gp = attention_group_planes(B, L, h_kv);
+    if (many && gp >= BH) {
+        // Many items per CTA and every plane's K' and V fit L2 together: the round-robin order, every other
+        // round reversed (snake), as lists.
+        lists.assign(grid, {});
+        for (int w = 0; w < total; ++w) {
+            const int r = w / grid, c = w % grid;
+            lists[(r & 1) ? grid - 1 - c : c].push_back(w);
+        }
+    } else if (many) {
+        // Many items per CTA: any dealing balances, so deal for L2 reuse instead.  The planes (b, u) are
+        // taken a group at a time (attention_group_planes), each group's items heaviest first to the least
+        // loaded CTA: every CTA runs through the groups in the same order, so the K' and V tiles read at
+        // any moment belong to one group or two and stay in L2.  With all planes at once the B=4, L=8192,
+        // 64/8-head workload read its K' and V from DRAM about six times over.
+        const int pairs = total / BH;
+        lists.assign(grid, {});
+        std::set<std::pair<long long, int>> bins;   // (load, cta)
+        for (int c = 0; c < grid; ++c) bins.insert({0, c});
+        std::vector<int> grp_items;
+        for (int g0 = 0; g0 < BH; g0 += gp) {
+            grp_items.clear();
+            for (int pr = 0; pr < pairs; ++pr)
+                for (int pl = g0; pl < std::min(BH, g0 + gp); ++pl) grp_items.push_back(pr * BH + pl);
+            std::stable_sort(grp_items.begin(), grp_items.end(), [&](int a, int b) { return cost[a] > cost[b]; });
+            for (int w : grp_items) {
+                auto it = bins.begin();   // the least loaded CTA
+                const auto [load, c] = *it;
+                bins.erase(it);
+                bins.insert({load + cost[w], c});
+                lists[c].push_back(w);
+            }
+        }
+    }
     csr.assign(static_cast<size_t>(grid) + 1 + total, 0);
     int at = 0;
     for (int c = 0; c < grid; ++c) {
@@ -289,23 +348,17 @@ bool plan_attention_schedule(int B, int L, int h_q, int h_kv, int grid, std::vec
         for (int w : lists[c]) csr[grid + 1 + at++] = w;
     }
     csr[grid] = at;
-    return 100 * snake_max <= 102 * cap;
+    return many && gp < BH;
 }
 
-int attention_schedule(DeviceState* st, const gqa::prefill::Params& p, int grid, bool* use_snake) {
+int attention_schedule(DeviceState* st, const gqa::prefill::Params& p, int grid) {
     const int key[5] = {p.B, p.L, p.h_q, p.h_kv, grid};
-    if (st->sched_valid && std::equal(key, key + 5, st->sched_key)) {
-        *use_snake = st->sched_snake;
-        return GQA_OK;
-    }
+    if (st->sched_valid && std::equal(key, key + 5, st->sched_key)) return GQA_OK;
     st->sched_valid = false;
     std::vector<int> csr;
-    const bool snake = plan_attention_schedule(p.B, p.L, p.h_q, p.h_kv, grid, csr);
+    plan_attention_schedule(p.B, p.L, p.h_q, p.h_kv, grid, csr);
     std::copy(key, key + 5, st->sched_key);
-    st->sched_snake = snake;
     st->sched_valid = true;
-    *use_snake = snake;
-    if (snake) return GQA_OK;
     const size_t bytes = csr.size() * sizeof(int);
     if (!ensure(st->sched, st->sched_bytes, bytes)) {
         st->sched_valid = false;
@@ -351,11 +404,10 @@ int launch_attention(DeviceState* st, const void* qr, const void* kr, const void
     p.total_work = static_cast<int>(total);
     // Persistent: one CTA per SM (each holds a whole SM's tensor memory), at most one per work item.
     const int grid = static_cast<int>(total < st->num_sms ? total : st->num_sms);
-    bool use_snake = true;
-    const int rc = attention_schedule(st, p, grid, &use_snake);
+    const int rc = attention_schedule(st, p, grid);
     if (rc != GQA_OK) return rc;
-    p.sched_start = use_snake ? nullptr : static_cast<const int*>(st->sched);
-    p.sched = use_snake ? nullptr : static_cast<const int*>(st->sched) + grid + 1;
+    p.sched_start = static_cast<const int*>(st->sched);
+    p.sched = static_cast<const int*>(st->sched) + grid + 1;
     bool& ready = st->attn_ready[D == 128 ? 1 : 0];
     if (!ready) {
         if (cudaFuncSetAttribute(attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, Layout<D>::DYN) !=
@@ -916,15 +968,15 @@ int gqa_last_error(void) {
 }
 
 int gqa_prefill_schedule(int B, int L, int h_q, int h_kv, int grid, int* starts, int* items, int capacity,
-                         int* snake) {
+                         int* grouped) {
     if (B <= 0 || L <= 0 || h_q <= 0 || h_kv <= 0 || h_q % h_kv != 0 || grid <= 0) return GQA_ERR_DIMS;
     const long long total = static_cast<long long>((L + 127) / 128 * (h_q / h_kv) + 1) / 2 * B * h_kv;
     if (total > 0x7fffffffLL || static_cast<long long>(B) * (h_q + h_kv) * 64 > 0x7fffffffLL || L > (1 << 30))
         return GQA_ERR_DIMS;
     const int g = total < grid ? static_cast<int>(total) : grid;
     std::vector<int> csr;
-    const bool use_snake = plan_attention_schedule(B, L, h_q, h_kv, g, csr);
-    if (snake) *snake = use_snake ? 1 : 0;
+    const bool by_group = plan_attention_schedule(B, L, h_q, h_kv, g, csr);
+    if (grouped) *grouped = by_group ? 1 : 0;
     if (starts && items && capacity >= total) {
         std::copy(csr.begin(), csr.begin() + g + 1, starts);
         std::copy(csr.begin() + g + 1, csr.end(), items);

@@ -90,7 +90,7 @@ struct Params {
     int total_work;            // tile pairs in all: ceil(tiles_per_group / 2) * B * h_kv
     float scale_log2;          // log2(e) / sqrt(D)
     // The work list of each CTA: items sched[sched_start[c] .. sched_start[c + 1]) for CTA c, in order
-    // (built on the host, see work_item); nullptr: the snake order below.
+    // (built on the host, see work_item).
     const int* sched_start;
     const int* sched;
     int* err;
@@ -282,16 +282,11 @@ __device__ __forceinline__ PairWork pair_work(const Params& p, int w) {
     return r;
 }
 
-// The r-th item of persistent CTA c out of G (p.total_work once the CTA's list is done).  With a host-built
-// schedule, the CTA's own list: the items dealt out by best fit, heaviest first, so that every CTA carries
-// about the same number of key tiles.  Without one: rounds of G consecutive items, every other round
-// reversed (snake order).
-__device__ __forceinline__ int work_item(const Params& p, int r, int c, int G) {
-    if (p.sched != nullptr) {
-        const int i = __ldg(p.sched_start + c) + r;
-        return i < __ldg(p.sched_start + c + 1) ? __ldg(p.sched + i) : p.total_work;
-    }
-    return r * G + ((r & 1) ? (G - 1 - c) : c);
+// The r-th item of persistent CTA c (p.total_work once the CTA's list is done): its own list, built on the
+// host so that every CTA carries about the same number of key tiles.
+__device__ __forceinline__ int work_item(const Params& p, int r, int c) {
+    const int i = __ldg(p.sched_start + c) + r;
+    return i < __ldg(p.sched_start + c + 1) ? __ldg(p.sched + i) : p.total_work;
 }
 
 template <int D>
@@ -306,7 +301,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int G = gridDim.x, cta = blockIdx.x;
+    const int cta = blockIdx.x;
 
     if (threadIdx.x == 0) {
         for (int k = 0; k < 2; ++k) {
@@ -363,7 +358,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         uint32_t o_seen = 0;   // PV_k products issued for the pairs handled so far (o_full phases)
         bool ok = true;
         for (int it = 0; ok; ++it) {
-            const int w = work_item(p, it, cta, G);
+            const int w = work_item(p, it, cta);
             if (w >= p.total_work) break;
             const PairWork pw = pair_work(p, w);
             const int nk = k ? pw.n1 : pw.n0;
@@ -470,7 +465,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             uint32_t kv = 0;                 // K/V tiles issued so far (ring position)
             bool ok = true;
             for (int it = 0; ok; ++it) {
-                const int w = work_item(p, it, cta, G);
+                const int w = work_item(p, it, cta);
                 if (w >= p.total_work) break;
                 const PairWork pw = pair_work(p, w);
                 const int n[2] = {pw.n0, pw.n1};
@@ -513,7 +508,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             uint32_t qn[2] = {0u, 0u};   // Q' tiles issued into buffer k so far
             bool ok = true;
             for (int it = 0; ok; ++it) {
-                const int w = work_item(p, it, cta, G);
+                const int w = work_item(p, it, cta);
                 if (w >= p.total_work) break;
                 const PairWork pw = pair_work(p, w);
                 for (int k = 0; k < 2 && ok; ++k) {
@@ -576,7 +571,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             uint32_t pn[2] = {0u, 0u};     // p_full phases consumed per tile
             bool ok = true;
             for (int it = 0; ok; ++it) {
-                const int w = __shfl_sync(0xffffffffu, work_item(p, it, cta, G), 0);
+                const int w = __shfl_sync(0xffffffffu, work_item(p, it, cta), 0);
                 if (w >= p.total_work) break;
                 const PairWork pw = pair_work(p, w);
                 const int n[2] = {pw.n0, pw.n1};

@@ -263,9 +263,12 @@ GQA_API int gqa_last_error(void);
  * The work items are pairs of 128-row query tiles of one (batch row, KV group): item w covers the tiles
  * 2(w / (B*h_kv)) and 2(w / (B*h_kv)) + 1 of the group b*h_kv + u = w mod (B*h_kv), whose tiles are listed
  * by query tile descending, then head ascending (causal masking: tile index i needs L/128 - i/g key tiles).
- * With more items than CTAs, the items are packed by best fit decreasing on (key tiles + a fixed
- * per-item cost), each CTA taking its items in the listed order; where the plain round-robin order is
- * within 2 % of that packing it is kept instead (*snake = 1) and the lists are those of the packing only.
+ * With more items than CTAs, each CTA takes its items in the listed order.  Where there are few items per
+ * CTA they are packed by best fit decreasing on (key tiles + a fixed per-item cost), for balance.  Where a
+ * plain round-robin order (every other round reversed) is already within 2 % of that packing, it is used
+ * as it is if the K' and V of all (b, u) planes fit in 48 MB (at d = 128), and otherwise (*grouped = 1) the
+ * items are dealt for L2 reuse: the planes a group at a time (as many as keep 16 MB of K' and V, at least
+ * one), each group's items heaviest first to the least loaded CTA.
  *   starts  [min(grid, items) + 1] CTA c's items are items[starts[c] .. starts[c+1])   (caller-owned)
  *   items   [items]                                                                   (caller-owned)
  *   capacity  the room in items; the arrays are written only when it suffices (and both are non-null)
@@ -273,7 +276,7 @@ GQA_API int gqa_last_error(void);
  * gqa_prefill rejects.
  */
 GQA_API int gqa_prefill_schedule(int B, int L, int h_q, int h_kv, int grid, int* starts, int* items, int capacity,
-                                 int* snake);
+                                 int* grouped);
 
 /* Frees the internal workspaces (and the cos / sin table) of every device this process used (synchronises each). */
 GQA_API void gqa_release(void);

@@ -46,8 +46,10 @@ def test_every_item_exactly_once_heaviest_first(B, L, h_q, h_kv):
     assert len(lists) == min(148, len(tiles))
     flat = np.concatenate([np.array(l, dtype=np.int64) for l in lists])
     assert np.array_equal(np.sort(flat), np.arange(len(tiles)))
-    for l in lists:
-        assert np.all(np.diff(tiles[l]) <= 0)   # each CTA takes its heaviest item first
+    _, grouped = G.prefill_schedule(B, L, h_q, h_kv, 148)
+    if not grouped:
+        for l in lists:
+            assert np.all(np.diff(tiles[l]) <= 0)   # each CTA takes its heaviest item first
 
 
 def test_packing_balances_the_headline_shape():
@@ -55,8 +57,8 @@ def test_packing_balances_the_headline_shape():
     mean number of key tiles; the packing is used there and its busiest CTA carries fewer key tiles."""
     B, L, h_q, h_kv = 1, 4096, 28, 4
     tiles = item_tiles(B, L, h_q, h_kv)
-    lists, snake = G.prefill_schedule(B, L, h_q, h_kv, 148)
-    assert not snake
+    lists, grouped = G.prefill_schedule(B, L, h_q, h_kv, 148)
+    assert not grouped
     packed = np.array([tiles[l].sum() for l in lists])
     rr = snake_loads(tiles, 148)
     assert rr.max() > 1.09 * tiles.sum() / 148
@@ -64,13 +66,41 @@ def test_packing_balances_the_headline_shape():
     assert packed.sum() == tiles.sum()
 
 
-@pytest.mark.parametrize("B,L,h_q,h_kv", [(1, 32768, 28, 4), (4, 8192, 64, 8), (1, 16384, 28, 4)])
-def test_round_robin_kept_where_already_balanced(B, L, h_q, h_kv):
+def group_planes(B, L, h_kv):
+    """Planes dealt together: K' and V of d = 128 within 16 MB, at least one, at most all."""
+    return max(1, min(B * h_kv, (16 << 20) // (2 * L * 128 * 2)))
+
+
+@pytest.mark.parametrize("B,L,h_q,h_kv", [(1, 16384, 28, 4), (2, 8192, 28, 4)])
+def test_many_items_round_robin_where_all_planes_fit_l2(B, L, h_q, h_kv):
+    """K' and V of all planes within 48 MB: the snake order, as lists."""
     tiles = item_tiles(B, L, h_q, h_kv)
-    _, snake = G.prefill_schedule(B, L, h_q, h_kv, 148)
-    assert snake
+    lists, grouped = G.prefill_schedule(B, L, h_q, h_kv, 148)
+    assert not grouped
+    for c, l in enumerate(lists):
+        expect = [w for w in range(len(tiles)) if (147 - w % 148 if (w // 148) & 1 else w % 148) == c]
+        assert l == expect
+
+
+@pytest.mark.parametrize("B,L,h_q,h_kv", [(1, 32768, 28, 4), (4, 8192, 64, 8)])
+def test_many_items_dealt_by_plane_group_and_balanced(B, L, h_q, h_kv):
+    """Where round-robin would already balance (many items per CTA), the items are dealt plane group by
+    plane group for L2 reuse: every CTA's list runs through the groups in order, and the busiest CTA stays
+    within one item of the mean load (costs: key tiles + 4 per item)."""
+    tiles = item_tiles(B, L, h_q, h_kv)
+    lists, grouped = G.prefill_schedule(B, L, h_q, h_kv, 148)
+    assert grouped
     rr = snake_loads(tiles, 148)
-    assert rr.max() <= 1.01 * tiles.sum() / 148 + tiles.max()
+    assert rr.max() <= 1.01 * tiles.sum() / 148 + tiles.max()   # the round-robin order was balanced too
+    planes, gp = B * h_kv, group_planes(B, L, h_kv)
+    cost = tiles + 4
+    loads = np.array([cost[l].sum() for l in lists])
+    assert loads.max() <= loads.mean() + cost.max()
+    for l in lists:
+        grp = (np.array(l) % planes) // gp
+        assert np.all(np.diff(grp) >= 0)                       # groups in order
+        for g in np.unique(grp):                                # heaviest first within a group
+            assert np.all(np.diff(tiles[np.array(l)[grp == g]]) <= 0)
 
 
 def test_fewer_items_than_ctas():
