@@ -338,7 +338,7 @@ def config_entry(w, *, world, step_ms, attn_ms, peaks, peak_src, cpu_base):
 
 def build_line(*, world, K, W, only, do_p, do_d, wp, wd, value_tflops, pre_mean, attn_mean, dec_mean, split_mean,
                total_rows, page, peaks, peak_src, cpu_base, e2e_pre, e2e_dec, pre_io, dec_io, qkv_line, clocks,
-               t_wall, configs=None):
+               t_wall, configs=None, dec_alone=(float("nan"), float("nan"))):
     """The JSON line of the `ours` arm from the measured numbers (no device work, so the CPU tests cover it).
     Times in ms; pre_io / dec_io = (host->device, device->host) bytes of one end-to-end prefill / decode
     step; a leg that did not run carries NaN, which clean() turns into null."""
@@ -375,7 +375,8 @@ def build_line(*, world, K, W, only, do_p, do_d, wp, wd, value_tflops, pre_mean,
         "e2e": {"value": world * fl / (e2e_pre * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "h2d_bytes_per_step": pre_io[0], "d2h_bytes_per_step": pre_io[1]},
         "gpu_launches": (2 * do_p + 3 * do_d) * 2 * K + (6 * K if qkv_line else 0)
-                        + 2 * 2 * K * sum(1 for n in (configs or {}) if n != wp.name),
+                        + 2 * 2 * K * sum(1 for n in (configs or {}) if n != wp.name)
+                        + (3 * 2 * K if dec_alone[0] == dec_alone[0] else 0),
         "qkv": qkv_line,
         "clocks": clocks,
         "decode": {
@@ -390,6 +391,11 @@ def build_line(*, world, K, W, only, do_p, do_d, wp, wd, value_tflops, pre_mean,
                          "peak_source": f"{peak_src} HBM copy",
                          "traffic": profile_traffic("split_kernel", DECODE_WORKLOAD + (f"-paged{page}" if page else "")),
                          "algorithmic_bytes_per_launch": allb, "ms_per_launch": split_mean},
+            "alone": {"ms_per_step": dec_alone[0], "value": world * allb / (dec_alone[0] * 1e-3) / 1e9, "unit": "GB/s",
+                      "split_ms_per_launch": dec_alone[1],
+                      "split_frac": allb / (dec_alone[1] * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                      "note": "the same decode in steps of its own (L2 flushed before each), not right after "
+                              "the long prefill"},
             "e2e": {"value": world * allb / (e2e_dec * 1e-3) / 1e9, "unit": "GB/s",
                     "h2d_bytes_per_step": dec_io[0], "d2h_bytes_per_step": dec_io[1],
                     "note": "the KV cache is resident device state; the step's inputs are q, the lengths"
@@ -509,6 +515,31 @@ def run_ours(args):
     dec_mean = reduce_max(sum(dec_ms) / K, dev)
     attn_mean = sum(attn_ms) / K
     split_mean = sum(split_ms) / K
+
+    # ---- the decode alone: K steps of decode only (L2 flushed before each), beside the in-step figure.
+    # Right after the long prefill the same decode runs ~20 % slower (measured: also after 2 ms idle, and
+    # with L2 left clean), so the step's decode half is reported as measured and this one beside it.
+    dec_alone_ms = split_alone_ms = float("nan")
+    if do_d and do_p:
+        for _ in range(W):
+            flush.zero_()
+            dec_call(qd, s, table)
+        da = [[ev() for _ in range(4)] for _ in range(K)]
+        torch.cuda.synchronize()
+        barrier()
+        for i in range(K):
+            flush.zero_()
+            da[i][0].record()
+            dec_call(qd, s, table)
+            da[i][3].record()
+            flush.zero_()
+            G.set_timing_events(da[i][1], da[i][2])
+            dec_call(qd, s, table)
+            G.set_timing_events(None, None)
+        torch.cuda.synchronize()
+        barrier()
+        dec_alone_ms = reduce_max(sum(e[0].elapsed_time(e[3]) for e in da) / K, dev)
+        split_alone_ms = sum(e[1].elapsed_time(e[2]) for e in da) / K
 
     # ---- end to end through the public API: pinned host inputs in, host result out, every step
     run_e2e = not args.no_e2e and do_p and do_d
@@ -645,7 +676,8 @@ def run_ours(args):
             e2e_pre=e2e_pre, e2e_dec=e2e_dec,
             pre_io=(sum(x.numel() * x.element_size() for x in (q, k, v)), out.numel() * out.element_size()),
             dec_io=(qd.numel() * 2 + s.numel() * 4 + (table.numel() * 4 if page else 0), outd.numel() * 2),
-            qkv_line=qkv_line, clocks=sampler.summary(), t_wall=t_wall, configs=configs)
+            qkv_line=qkv_line, clocks=sampler.summary(), t_wall=t_wall, configs=configs,
+            dec_alone=(dec_alone_ms, split_alone_ms))
     if torch.distributed.is_initialized():
         barrier()
         torch.distributed.destroy_process_group()

@@ -16,7 +16,7 @@ CONTRACT = ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step
             "impl")
 
 
-def line_for(only, world=1, page=None, qkv=None, configs=None):
+def line_for(only, world=1, page=None, qkv=None, configs=None, dec_alone=(NAN, NAN)):
     do_p, do_d = only in (None, "prefill"), only in (None, "decode")
     wp, wd = gi.BY_NAME[bench.PREFILL_WORKLOAD], gi.BY_NAME[bench.DECODE_WORKLOAD]
     fl = bench.prefill_flops(wp)
@@ -30,7 +30,7 @@ def line_for(only, world=1, page=None, qkv=None, configs=None):
         cpu_base={"value": 0.03, "unit": "TFLOP/s", "cores": 16, "kind": "oracle", "sample": "s"} if do_p else None,
         e2e_pre=1.3 if do_p else NAN, e2e_dec=0.4 if do_d else NAN, pre_io=(37748736, 29360128),
         dec_io=(459008, 458752), qkv_line=qkv, clocks={"sm_mhz": 1965, "sm_max_mhz": 1965, "reasons": []},
-        t_wall=0.05, configs=configs)
+        t_wall=0.05, configs=configs, dec_alone=dec_alone)
     text = json.dumps(bench.clean(line), allow_nan=False)   # strict JSON: no NaN or inf survives
     return json.loads(text)
 
@@ -103,3 +103,13 @@ def test_configs_carry_step_kernel_roofline_and_cpu_baseline():
     assert math.isclose(head["roofline"]["frac"], d["roofline"]["frac"])
     # two launches (rotation pass + attention) per step, two kinds of step, K steps, three more workloads
     assert d["gpu_launches"] == (2 + 3) * 2 * 30 + 3 * 2 * 2 * 30
+
+
+def test_decode_alone_beside_the_in_step_decode():
+    d = line_for(None, dec_alone=(0.345, 0.336))
+    a = d["decode"]["alone"]
+    allb = bench.decode_bytes(954557, gi.BY_NAME[bench.DECODE_WORKLOAD])
+    assert math.isclose(a["split_frac"], allb / 0.336e-3 / 1e9 / PEAKS["hbm_gbs"])
+    assert math.isclose(a["value"], allb / 0.345e-3 / 1e9)
+    assert d["gpu_launches"] == (2 + 3) * 2 * 30 + 3 * 2 * 30
+    assert line_for(None)["decode"]["alone"]["value"] is None   # not run: null, still strict JSON
