@@ -373,10 +373,13 @@ def build_line(*, world, K, W, only, do_p, do_d, wp, wd, value_tflops, pre_mean,
         "cpu_baseline": cpu_base,
         "only": only,
         "e2e": {"value": world * fl / (e2e_pre * 1e-3) / 1e12, "unit": "TFLOP/s",
-                "h2d_bytes_per_step": pre_io[0], "d2h_bytes_per_step": pre_io[1]},
+                "h2d_bytes_per_step": pre_io[0], "d2h_bytes_per_step": pre_io[1], "ms_per_step": e2e_pre,
+                "note": "steps pipelined over three streams (copy in, gqa_prefill, copy out) with two buffer "
+                        "sets; every step copies its own inputs in and its output out"},
         "gpu_launches": (2 * do_p + 3 * do_d) * 2 * K + (6 * K if qkv_line else 0)
                         + 2 * 2 * K * sum(1 for n in (configs or {}) if n != wp.name)
-                        + (3 * 2 * K if dec_alone[0] == dec_alone[0] else 0),
+                        + (3 * 2 * K if dec_alone[0] == dec_alone[0] else 0)
+                        + ((2 + 3) * K if e2e_pre == e2e_pre else 0),
         "qkv": qkv_line,
         "clocks": clocks,
         "decode": {
@@ -541,47 +544,77 @@ def run_ours(args):
         dec_alone_ms = reduce_max(sum(e[0].elapsed_time(e[3]) for e in da) / K, dev)
         split_alone_ms = sum(e[1].elapsed_time(e[2]) for e in da) / K
 
-    # ---- end to end through the public API: pinned host inputs in, host result out, every step
+    # ---- end to end through the public API: every step copies its inputs in from pinned host memory, runs
+    # the call and copies its result out to pinned host memory.  The prefill steps are pipelined as a
+    # serving process would run them: copies in on one stream, the call on another, copies out on a third,
+    # with two sets of device buffers, so step i+1's inputs travel while step i computes and step i-1's
+    # output travels back.  The rate is taken over K steps in steady state (after W), from the output copy
+    # of step W-1 to that of step W+K-1.  The decode steps (inputs and outputs of a few hundred KB) run one
+    # after another on one stream.
     run_e2e = not args.no_e2e and do_p and do_d
+    e2e_pre = e2e_dec = float("nan")
     if run_e2e:
         qh, kh, vh = (x.cpu().pin_memory() for x in (q, k, v))
-        outh = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        outh = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(2)]
+        dins = [tuple(torch.empty_like(x) for x in (q, k, v)) for _ in range(2)]
+        douts = [torch.empty_like(out) for _ in range(2)]
+        s_in, s_cmp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+        n = W + K
+        ev_in = [torch.cuda.Event() for _ in range(n)]
+        ev_cmp = [torch.cuda.Event() for _ in range(n)]
+        ev_out = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+        torch.cuda.synchronize()
+        barrier()
+        for i in range(n):
+            j = i & 1
+            with torch.cuda.stream(s_in):
+                if i >= 2:
+                    s_in.wait_event(ev_cmp[i - 2])        # buffer set j no longer read
+                for dst, src in zip(dins[j], (qh, kh, vh)):
+                    dst.copy_(src, non_blocking=True)
+                ev_in[i].record(s_in)
+            with torch.cuda.stream(s_cmp):
+                s_cmp.wait_event(ev_in[i])
+                if i >= 2:
+                    s_cmp.wait_event(ev_out[i - 2])       # output buffer j copied out
+                G.prefill(*dins[j], theta=wp.theta, out=douts[j])
+                ev_cmp[i].record(s_cmp)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_cmp[i])
+                outh[j].copy_(douts[j], non_blocking=True)
+                ev_out[i].record(s_out)
+        torch.cuda.synchronize()
+        barrier()
+        e2e_pre = reduce_max(ev_out[W - 1].elapsed_time(ev_out[W + K - 1]) / K, dev)
+
         qdh, sh_ = qd.cpu().pin_memory(), s.cpu().pin_memory()
         outdh = torch.empty(outd.shape, dtype=outd.dtype).pin_memory()
-        qx, kx, vx, qdx, sx = (torch.empty_like(x) for x in (q, k, v, qd, s))
+        qdx, sx = torch.empty_like(qd), torch.empty_like(s)
         th = table.cpu().pin_memory() if table is not None else None
         tx = torch.empty_like(table) if table is not None else None
 
-    def e2e_step(e):
-        flush.zero_()
-        e[0].record()
-        qx.copy_(qh, non_blocking=True)
-        kx.copy_(kh, non_blocking=True)
-        vx.copy_(vh, non_blocking=True)
-        G.prefill(qx, kx, vx, theta=wp.theta, out=out)
-        outh.copy_(out, non_blocking=True)
-        e[1].record()
-        qdx.copy_(qdh, non_blocking=True)
-        sx.copy_(sh_, non_blocking=True)
-        if tx is not None:
-            tx.copy_(th, non_blocking=True)
-        dec_call(qdx, sx, tx)
-        outdh.copy_(outd, non_blocking=True)
-        e[2].record()
+        def e2e_dec_step(e):
+            flush.zero_()
+            e[0].record()
+            qdx.copy_(qdh, non_blocking=True)
+            sx.copy_(sh_, non_blocking=True)
+            if tx is not None:
+                tx.copy_(th, non_blocking=True)
+            dec_call(qdx, sx, tx)
+            outdh.copy_(outd, non_blocking=True)
+            e[1].record()
 
-    e2e_pre = e2e_dec = float("nan")
-    if run_e2e:
         for _ in range(max(1, W)):
-            e2e_step([ev() for _ in range(3)])
-        e2e_evs = [[ev() for _ in range(3)] for _ in range(K)]
+            e2e_dec_step([ev() for _ in range(2)])
+        e2e_evs = [[ev() for _ in range(2)] for _ in range(K)]
         torch.cuda.synchronize()
         barrier()
         for i in range(K):
-            e2e_step(e2e_evs[i])
+            e2e_dec_step(e2e_evs[i])
         torch.cuda.synchronize()
         barrier()
-        e2e_pre = reduce_max(sum(e[0].elapsed_time(e[1]) for e in e2e_evs) / K, dev)
-        e2e_dec = reduce_max(sum(e[1].elapsed_time(e[2]) for e in e2e_evs) / K, dev)
+        e2e_dec = reduce_max(sum(e[0].elapsed_time(e[1]) for e in e2e_evs) / K, dev)
+        del dins, douts, outh
 
     # ---- the fused route from hidden states: QKV projection + bias + RoPE (writing Q', K' and the cache
     # rows K, V), then the attention on the rotated inputs -- no prep pass.  Timed like the headline

@@ -45,7 +45,7 @@ def test_both_halves():
     assert math.isclose(r["frac"], r["achieved"] / PEAKS["bf16_tflops"])
     dr = d["decode"]["roofline"]
     assert dr["bound"] == "hbm" and math.isclose(dr["frac"], dr["achieved"] / PEAKS["hbm_gbs"])
-    assert d["gpu_launches"] == (2 + 3) * 2 * 30
+    assert d["gpu_launches"] == (2 + 3) * 2 * 30 + (2 + 3) * 30   # headline + kernel-timing steps, e2e steps
     assert d["e2e"]["h2d_bytes_per_step"] == 37748736 and d["decode"]["e2e"]["d2h_bytes_per_step"] == 458752
     assert d["impl"] == "ours" and d["scaling"] == "weak"
 
@@ -54,7 +54,7 @@ def test_only_prefill_drops_the_decode_half():
     d = line_for("prefill")
     assert d["decode"] is None
     assert d["value"] > 0 and d["roofline"]["frac"] > 0
-    assert d["gpu_launches"] == 2 * 2 * 30
+    assert d["gpu_launches"] == 2 * 2 * 30 + (2 + 3) * 30
 
 
 def test_only_decode_carries_no_prefill_figures():
@@ -102,7 +102,7 @@ def test_configs_carry_step_kernel_roofline_and_cpu_baseline():
     head = d["configs"][bench.PREFILL_WORKLOAD]
     assert math.isclose(head["roofline"]["frac"], d["roofline"]["frac"])
     # two launches (rotation pass + attention) per step, two kinds of step, K steps, three more workloads
-    assert d["gpu_launches"] == (2 + 3) * 2 * 30 + 3 * 2 * 2 * 30
+    assert d["gpu_launches"] == (2 + 3) * 2 * 30 + 3 * 2 * 2 * 30 + (2 + 3) * 30
 
 
 def test_decode_alone_beside_the_in_step_decode():
@@ -111,5 +111,5 @@ def test_decode_alone_beside_the_in_step_decode():
     allb = bench.decode_bytes(954557, gi.BY_NAME[bench.DECODE_WORKLOAD])
     assert math.isclose(a["split_frac"], allb / 0.336e-3 / 1e9 / PEAKS["hbm_gbs"])
     assert math.isclose(a["value"], allb / 0.345e-3 / 1e9)
-    assert d["gpu_launches"] == (2 + 3) * 2 * 30 + 3 * 2 * 30
+    assert d["gpu_launches"] == (2 + 3) * 2 * 30 + 3 * 2 * 30 + (2 + 3) * 30
     assert line_for(None)["decode"]["alone"]["value"] is None   # not run: null, still strict JSON
