@@ -286,7 +286,7 @@ def measure_prefill(G, w, K: int, W: int, flush, dev):
     """Time gqa_prefill on workload w: W warm-up steps, then K headline steps (no per-kernel events, so
     the attention kernel stays a programmatic dependent of the rotation pass) interleaved with K steps
     that record events around the attention kernel alone; the L2 is flushed before every step.
-    Returns (mean step ms, max over ranks; mean attention-kernel ms on this rank)."""
+    Returns (mean step ms, max over ranks; mean attention-kernel ms on this rank; wall seconds of the loop)."""
     q, k, v = gi.prefill_inputs(w, device=str(dev))
     out = torch.empty_like(q)
 
@@ -306,34 +306,52 @@ def measure_prefill(G, w, K: int, W: int, flush, dev):
     kevs = [[ev() for _ in range(4)] for _ in range(K)]
     torch.cuda.synchronize()
     barrier()
+    t0 = time.perf_counter()
     for i in range(K):
         step(evs[i], False)
         step(kevs[i], True)
     torch.cuda.synchronize()
+    wall = time.perf_counter() - t0
     barrier()
     if G.last_error() != 0:
         raise RuntimeError(f"device error while timing {w.name}")
     step_ms = reduce_max(sum(e[0].elapsed_time(e[3]) for e in evs) / K, dev)
     attn_ms = sum(e[1].elapsed_time(e[2]) for e in kevs) / K
     del q, k, v, out
-    return step_ms, attn_ms
+    return step_ms, attn_ms, wall
 
 
-def config_entry(w, *, world, step_ms, attn_ms, peaks, peak_src, cpu_base):
+LONG_RUN_S = 0.1   # a timed loop this long under the power cap counts as "a kernel timed inside a long step"
+
+
+def tensor_peak(peaks, clocks, wall_s):
+    """The bf16 peak a tensor-bound kernel is measured against: the measured burst figure for a kernel timed
+    alone, the measured sustained figure (cuBLAS back to back for seconds, under the 1 kW power cap) for a
+    kernel timed inside a long run whose clock record shows the power cap active."""
+    capped = isinstance(clocks, dict) and "sw_power_cap" in (clocks.get("reasons") or [])
+    if capped and wall_s == wall_s and wall_s >= LONG_RUN_S:
+        return peaks["bf16_tflops_sustained"], "sustained"
+    return peaks["bf16_tflops"], "burst"
+
+
+def config_entry(w, *, world, step_ms, attn_ms, peaks, peak_src, cpu_base, clocks=None, wall_s=float("nan")):
     """The `configs` entry of one prefill workload from its measured step and kernel times (ms)."""
     fl = prefill_flops(w)
     step_t = fl / (step_ms * 1e-3) / 1e12
     ach = fl / (attn_ms * 1e-3) / 1e12
+    peak, kind = tensor_peak(peaks, clocks, wall_s)
     return {"workload": w.desc, "B": w.B, "L": w.L, "h_q": w.h_q, "h_kv": w.h_kv, "d": w.d,
             "value": world * step_t, "unit": "TFLOP/s", "ms_per_step": step_ms,
             "step_frac": step_t / peaks["bf16_tflops"],
             "kernel_ms_per_launch": attn_ms,
             "roofline": {"kernel": "attn_kernel (prefill)", "bound": "tensor", "achieved": ach,
-                         "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": ach / peaks["bf16_tflops"],
-                         "peak_source": f"{peak_src} bf16 dense (burst)",
+                         "peak": peak, "unit": "TFLOP/s", "frac": ach / peak,
+                         "peak_source": f"{peak_src} bf16 dense ({kind})",
+                         "frac_of_burst": ach / peaks["bf16_tflops"],
+                         "frac_of_sustained": ach / peaks["bf16_tflops_sustained"],
                          "traffic": profile_traffic("attn_kernel", w.name),
                          "algorithmic_flops_per_launch": fl, "ms_per_launch": attn_ms},
-            "cpu_baseline": cpu_base}
+            "cpu_baseline": cpu_base, "clocks": clocks, "wall_s_timed_region": wall_s}
 
 
 def build_line(*, world, K, W, only, do_p, do_d, wp, wd, value_tflops, pre_mean, attn_mean, dec_mean, split_mean,
@@ -347,6 +365,7 @@ def build_line(*, world, K, W, only, do_p, do_d, wp, wd, value_tflops, pre_mean,
     allb = decode_bytes(total_rows, wd)
     # --only decode: attn_mean is NaN, and the prefill roofline below is dropped from the line
     achieved_t = fl / (attn_mean * 1e-3) / 1e12
+    peak_t, peak_kind = tensor_peak(peaks, clocks, t_wall)
     achieved_b = allb / (split_mean * 1e-3) / 1e9
     line = {
         "metric": METRIC,
@@ -360,12 +379,15 @@ def build_line(*, world, K, W, only, do_p, do_d, wp, wd, value_tflops, pre_mean,
                        timing=f"{K} headline steps without per-kernel events, interleaved with {K} steps "
                               "with CUDA events around the attention / split kernels for the roofline"),
         "roofline": {"kernel": "attn_kernel (prefill)", "bound": "tensor", "achieved": achieved_t,
-                     "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved_t / peaks["bf16_tflops"],
-                     "peak_source": f"{peak_src} bf16 dense (burst)",
+                     "peak": peak_t, "unit": "TFLOP/s", "frac": achieved_t / peak_t,
+                     "peak_source": f"{peak_src} bf16 dense ({peak_kind}: "
+                                    + ("timed inside a long run with the power cap active)" if peak_kind == "sustained"
+                                       else "no long power-capped run)"),
                      "traffic": profile_traffic("attn_kernel", wp.name),
                      "algorithmic_flops_per_launch": fl, "ms_per_launch": attn_mean,
-                     # beside the burst peak: the sustained cuBLAS figure and the 2.25 PFLOP/s data-sheet
-                     # number, and the exponentials per launch (one per unmasked score)
+                     # both measured peaks, the 2.25 PFLOP/s data-sheet number, and the exponentials per
+                     # launch (one per unmasked score)
+                     "frac_of_burst": achieved_t / peaks["bf16_tflops"],
                      "frac_of_sustained": achieved_t / peaks["bf16_tflops_sustained"],
                      "frac_of_spec": achieved_t / SPEC_BF16_TFLOPS,
                      "exp_per_launch": wp.B * wp.h_q * wp.L * (wp.L + 1) // 2,
@@ -408,7 +430,8 @@ def build_line(*, world, K, W, only, do_p, do_d, wp, wd, value_tflops, pre_mean,
         "impl": "ours",
         # every prefill workload: the headline's own figures, then the others timed after it
         "configs": dict({wp.name: config_entry(wp, world=world, step_ms=pre_mean, attn_ms=attn_mean, peaks=peaks,
-                                               peak_src=peak_src, cpu_base=cpu_base)} if do_p else {},
+                                               peak_src=peak_src, cpu_base=cpu_base, clocks=clocks,
+                                               wall_s=t_wall)} if do_p else {},
                         **(configs or {})),
     }
     if not do_p:   # --only decode: the line carries the decode half alone
@@ -696,11 +719,10 @@ def run_ours(args):
     for name in names:
         wc = gi.BY_NAME[name]
         with ClockSampler(local) as c_clk:
-            c_step, c_attn = measure_prefill(G, wc, K, W, flush, dev)
+            c_step, c_attn, c_wall = measure_prefill(G, wc, K, W, flush, dev)
         c_cpu = cpu_baseline(wc, budget_s=4.0) if (rank == 0 and world == 1 and not args.no_cpu_baseline) else None
         configs[name] = config_entry(wc, world=world, step_ms=c_step, attn_ms=c_attn, peaks=peaks,
-                                     peak_src=peak_src, cpu_base=c_cpu)
-        configs[name]["clocks"] = c_clk.summary()
+                                     peak_src=peak_src, cpu_base=c_cpu, clocks=c_clk.summary(), wall_s=c_wall)
     line = None
     if rank == 0:
         line = build_line(

@@ -113,3 +113,19 @@ def test_decode_alone_beside_the_in_step_decode():
     assert math.isclose(a["value"], allb / 0.345e-3 / 1e9)
     assert d["gpu_launches"] == (2 + 3) * 2 * 30 + 3 * 2 * 30 + (2 + 3) * 30
     assert line_for(None)["decode"]["alone"]["value"] is None   # not run: null, still strict JSON
+
+
+def test_peak_is_sustained_only_for_long_power_capped_runs():
+    capped = {"sm_mhz": 1605, "sm_max_mhz": 1965, "reasons": ["sw_power_cap"]}
+    assert bench.tensor_peak(PEAKS, capped, 0.4) == (PEAKS["bf16_tflops_sustained"], "sustained")
+    assert bench.tensor_peak(PEAKS, capped, 0.01) == (PEAKS["bf16_tflops"], "burst")        # too short
+    assert bench.tensor_peak(PEAKS, {"reasons": []}, 0.4) == (PEAKS["bf16_tflops"], "burst")  # no cap
+    assert bench.tensor_peak(PEAKS, {"error": "nvml unavailable"}, 0.4) == (PEAKS["bf16_tflops"], "burst")
+    w = gi.BY_NAME["qwen2-72b-prefill-B4-L8192"]
+    c = bench.config_entry(w, world=1, step_ms=4.0, attn_ms=3.75, peaks=PEAKS, peak_src="measured", cpu_base=None,
+                           clocks=capped, wall_s=0.25)
+    ach = bench.prefill_flops(w) / 3.75e-3 / 1e12
+    r = c["roofline"]
+    assert r["peak"] == PEAKS["bf16_tflops_sustained"] and math.isclose(r["frac"], ach / r["peak"])
+    assert math.isclose(r["frac_of_burst"], ach / PEAKS["bf16_tflops"])
+    assert "sustained" in r["peak_source"]
