@@ -141,9 +141,6 @@ __global__ void __launch_bounds__(PREP_THREADS, GQA_PREP_MIN_CTAS) prep_kernel(c
     // distinct banks (lanes of the same chunk read the same address).
     constexpr int TROW4 = H / 2 + H / 8;
     __shared__ float4 tab[PREP_POS * TROW4];
-    // The attention kernel launched after this one may be scheduled now; it waits for this grid's
-    // results (griddepcontrol.wait) before reading Q' or K'.
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     __shared__ double finv[H];
     const int p0 = blockIdx.x * PREP_POS;
     const int heads = h_q + h_kv;
@@ -336,9 +333,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    // Q' and K' come from the prep kernel just before this one (programmatic dependent launch): wait for
-    // that grid to complete and its writes to be visible.  A no-op for a plain launch.
-    asm volatile("griddepcontrol.wait;" ::: "memory");
     const uint32_t tmem = sh.tmem_base;
     volatile int* abort = &sh.abort;
 
