@@ -10,7 +10,7 @@ over the Qwen2-7B-shaped decode workload (B=64 sequences, cache lengths uniform 
 headline `value` is the prefill's causal-effective TFLOP/s (4*B*h_q*d*L(L+1)/2 per step, summed over
 ranks, divided by the slowest rank's device time); the decode step is reported beside it in GB/s of KV
 cache.  The other prefill workloads (Qwen2-0.5B L=128, Qwen2-7B L=4096, Qwen2-72B B=4 L=8192) are timed
-the same way after the headline and reported under `configs`, each with its step and kernel times, its
+the same way before the headline and reported under `configs`, each with its step and kernel times, its
 roofline fraction and a CPU-oracle sample.  Inputs are synthetic (seeded N(0,1) bf16, drawn on the
 device) and resident in HBM when the timed region starts; the L2 is flushed (a 256 MiB write) before
 every prefill, and the decode cache (~2.1 GB) is far larger than L2.  Each rank of an N-GPU run
@@ -44,7 +44,7 @@ import gqa_inputs as gi  # noqa: E402
 
 METRIC = "GQA prefill TFLOP/s & decode KV GB/s, as % of B200 tensor/HBM peak"
 PREFILL_WORKLOAD = "qwen2-7b-prefill-L32768"   # the largest prefill workload that fits one GPU
-# The other prefill workloads, each timed after the headline and reported under `configs`.
+# The other prefill workloads, each timed before the headline and reported under `configs`.
 CONFIG_WORKLOADS = ("qwen2-0.5b-prefill-L128", "qwen2-7b-prefill-L4096", "qwen2-72b-prefill-B4-L8192")
 DECODE_WORKLOAD = "qwen2-7b-decode-B64"
 FLUSH_BYTES = 256 << 20
@@ -428,7 +428,7 @@ def build_line(*, world, K, W, only, do_p, do_d, wp, wd, value_tflops, pre_mean,
         },
         "wall_s_timed_region": t_wall,
         "impl": "ours",
-        # every prefill workload: the headline's own figures, then the others timed after it
+        # every prefill workload: the headline's own figures, then the others (timed before it)
         "configs": dict({wp.name: config_entry(wp, world=world, step_ms=pre_mean, attn_ms=attn_mean, peaks=peaks,
                                                peak_src=peak_src, cpu_base=cpu_base, clocks=clocks,
                                                wall_s=t_wall)} if do_p else {},
@@ -510,10 +510,24 @@ def run_ours(args):
         dec_alone_ms = reduce_max(sum(e[0].elapsed_time(e[3]) for e in da) / K, dev)
         split_alone_ms = sum(e[1].elapsed_time(e[2]) for e in da) / K
 
+    peaks, peak_src = load_peaks()
+    # ---- the other prefill workloads, one after another (each rank its own copy), each with its own
+    # step and kernel times, roofline fraction and (rank 0 of a 1-GPU run) a bounded CPU-oracle sample.
+    # Timed before the headline, like the decode alone: after seconds of the long prefill the GPU runs
+    # its short workloads at a lower SM clock under the power cap (L=4096: ~1790 against 1965 MHz).
+    configs = {}
+    names = [] if args.configs in ("", "none") or not do_p else [n for n in args.configs.split(",") if n != wp.name]
+    for name in names:
+        wc = gi.BY_NAME[name]
+        with ClockSampler(local) as c_clk:
+            c_step, c_attn, c_wall = measure_prefill(G, wc, K, W, flush, dev)
+        c_cpu = cpu_baseline(wc, budget_s=4.0) if (rank == 0 and world == 1 and not args.no_cpu_baseline) else None
+        configs[name] = config_entry(wc, world=world, step_ms=c_step, attn_ms=c_attn, peaks=peaks,
+                                     peak_src=peak_src, cpu_base=c_cpu, clocks=c_clk.summary(), wall_s=c_wall)
+
     def step(evs=None, inner=False):
-        """One step; with `inner` the library also records events around its main kernels, which makes
-        the attention launch a plain one (no overlap with the prep kernel), so the headline steps run
-        without them and separate steps time the kernels."""
+        """One step; with `inner` the library also records events around its main kernels (separate steps
+        time the kernels, so the headline steps carry no events between the prep and attention kernels)."""
         flush.zero_()
         if evs:
             evs[0].record()
@@ -711,18 +725,6 @@ def run_ours(args):
         }
         del xq, wqkv, bqkv, qo, w_o, x_in, y_out
 
-    peaks, peak_src = load_peaks()
-    # ---- the other prefill workloads, one after another (each rank its own copy), each with its own
-    # step and kernel times, roofline fraction and (rank 0 of a 1-GPU run) a bounded CPU-oracle sample
-    configs = {}
-    names = [] if args.configs in ("", "none") or not do_p else [n for n in args.configs.split(",") if n != wp.name]
-    for name in names:
-        wc = gi.BY_NAME[name]
-        with ClockSampler(local) as c_clk:
-            c_step, c_attn, c_wall = measure_prefill(G, wc, K, W, flush, dev)
-        c_cpu = cpu_baseline(wc, budget_s=4.0) if (rank == 0 and world == 1 and not args.no_cpu_baseline) else None
-        configs[name] = config_entry(wc, world=world, step_ms=c_step, attn_ms=c_attn, peaks=peaks,
-                                     peak_src=peak_src, cpu_base=c_cpu, clocks=c_clk.summary(), wall_s=c_wall)
     line = None
     if rank == 0:
         line = build_line(
@@ -757,7 +759,7 @@ def main(argv=None):
     ap.add_argument("--prefill-workload", default=PREFILL_WORKLOAD, choices=[w.name for w in gi.WORKLOADS if w.kind == "prefill"],
                     help="prefill workload of the step (default: the Qwen2-7B L=32768 headline workload)")
     ap.add_argument("--configs", default=",".join(CONFIG_WORKLOADS),
-                    help="comma list of further prefill workloads timed after the headline and reported under "
+                    help="comma list of further prefill workloads timed before the headline and reported under "
                          "`configs` ('none' for none)")
     ap.add_argument("--no-qkv", action="store_true", help="skip the fused QKV projection leg")
     ap.add_argument("--decode-page-size", type=int, default=None,
