@@ -202,8 +202,13 @@ def prefill_rows_ref(q, k, v, theta: float, b: int, t: int, rows) -> np.ndarray:
     return a @ as_f64(v[b, :n, u, :])
 
 
-def decode_one_ref(q_b, krows, vrows, theta: float, include_self: bool = False) -> np.ndarray:
-    """One sequence: q_b [h_q,d], cache rows krows/vrows [s,h_kv,d] -> float64 [h_q,d]."""
+def decode_one_ref(q_b, krows, vrows, theta: float, include_self: bool = False,
+                   k_rotated: bool = False) -> np.ndarray:
+    """One sequence: q_b [h_q,d], cache rows krows/vrows [s,h_kv,d] -> float64 [h_q,d].
+
+    The cached keys are raw projections, rotated here at their positions 0 .. s-1; with ``k_rotated`` they
+    already hold rope(k) at those positions (a cache that keeps the keys after RoPE) and are used as they
+    are.  The query is rotated at its position either way."""
     q_b = as_f64(q_b)
     krows = as_f64(krows)
     vrows = as_f64(vrows)
@@ -212,7 +217,7 @@ def decode_one_ref(q_b, krows, vrows, theta: float, include_self: bool = False) 
     g = h_q // h_kv
     p = s - 1 if include_self else s
     qr = rope(q_b[None, :, :], [p], theta)[0]
-    kr = rope(krows, np.arange(s), theta)
+    kr = krows if k_rotated else rope(krows, np.arange(s), theta)
     out = np.empty((h_q, d), dtype=np.float64)
     for t in range(h_q):
         u = head_group(t, g)
@@ -228,8 +233,9 @@ def packed_offsets(seqlens) -> np.ndarray:
 
 
 def decode_ref(q, kcache, vcache, seqlens, theta: float, include_self: bool = False,
-               batch_rows=None) -> np.ndarray:
-    """Decode step over the packed cache.  q [B,h_q,d]; caches [sum(seqlens),h_kv,d].
+               batch_rows=None, k_rotated: bool = False) -> np.ndarray:
+    """Decode step over the packed cache.  q [B,h_q,d]; caches [sum(seqlens),h_kv,d] (keys raw, or already
+    rotated at their positions with ``k_rotated``, as in decode_one_ref).
 
     Returns float64 [B,h_q,d], or [len(batch_rows),h_q,d] for a subset of sequences.
     """
@@ -239,17 +245,17 @@ def decode_ref(q, kcache, vcache, seqlens, theta: float, include_self: bool = Fa
     outs = []
     for b in bs:
         o0, o1 = int(off[b]), int(off[b + 1])
-        outs.append(decode_one_ref(q[b], kcache[o0:o1], vcache[o0:o1], theta, include_self))
+        outs.append(decode_one_ref(q[b], kcache[o0:o1], vcache[o0:o1], theta, include_self, k_rotated))
     return np.stack(outs, axis=0)
 
 
 def decode_paged_ref(q, kpages, vpages, block_table, seqlens, theta: float, batch_rows=None,
-                     include_self: bool = False) -> np.ndarray:
+                     include_self: bool = False, k_rotated: bool = False) -> np.ndarray:
     """Decode step over a paged cache (nxmr.cn page, §2.4: the cache of each KV head kept in blocks).
 
     kpages/vpages [num_pages, page_size, h_kv, d]; block_table [B, max_pages]: position j of sequence b is
     slot j % page_size of page block_table[b, j // page_size].  Gathers each sequence's rows in position
-    order and applies the decode definition of decode_one_ref (``include_self`` as there).
+    order and applies the decode definition of decode_one_ref (``include_self`` and ``k_rotated`` as there).
     """
     kp, vp, bt = np.asarray(kpages), np.asarray(vpages), np.asarray(block_table)
     page_size = kp.shape[1]
@@ -259,11 +265,12 @@ def decode_paged_ref(q, kpages, vpages, block_table, seqlens, theta: float, batc
     for b in bs:
         kr = np.stack([kp[bt[b, j // page_size], j % page_size] for j in range(seq[b])])
         vr = np.stack([vp[bt[b, j // page_size], j % page_size] for j in range(seq[b])])
-        outs.append(decode_one_ref(q[b], kr, vr, theta, include_self))
+        outs.append(decode_one_ref(q[b], kr, vr, theta, include_self, k_rotated))
     return np.stack(outs, axis=0)
 
 
-def qkv_append_ref(x, w_qkv, b_qkv, h_q: int, h_kv: int, d: int, seqlens, kpages, vpages, block_table):
+def qkv_append_ref(x, w_qkv, b_qkv, h_q: int, h_kv: int, d: int, seqlens, kpages, vpages, block_table,
+                   rotate_k: bool = False, theta=None):
     """One decode step's projection and cache append (aicoding.csdn.net page, §4.1.3 steps 1-2 and its
     closing paragraph: each step appends the current token's K and V to the cache of the h_kv groups;
     nxmr.cn page, §2.4: that cache kept in pages).
@@ -271,8 +278,9 @@ def qkv_append_ref(x, w_qkv, b_qkv, h_q: int, h_kv: int, d: int, seqlens, kpages
     x [B, d_model] is the new token of each sequence; its projection y = x w_qkv^T + b is split into
     q [B, h_q, d] and the rows k, v [B, h_kv, d].  The token sits at position p_b = seqlens[b] (the cache
     length before the append), so k and v go, un-rotated like every cache row, to slot p_b % page_size of
-    page block_table[b, p_b // page_size].  Returns (q float64 [B, h_q, d], un-rotated; the grown key and
-    value pages as float64 copies); the inputs are not modified.
+    page block_table[b, p_b // page_size]; with ``rotate_k`` (a cache that keeps keys after RoPE) k goes
+    there as rope(k) at p_b with base ``theta``.  Returns (q float64 [B, h_q, d], un-rotated; the grown key
+    and value pages as float64 copies); the inputs are not modified.
     """
     xf, wf = as_f64(x), as_f64(w_qkv)
     y = xf @ wf.T                                         # [B, (h_q + 2 h_kv) d]
@@ -288,7 +296,7 @@ def qkv_append_ref(x, w_qkv, b_qkv, h_q: int, h_kv: int, d: int, seqlens, kpages
     for b in range(B):
         pos = int(np.asarray(seqlens).reshape(-1)[b])
         page = int(bt[b, pos // page_size])
-        kp[page, pos % page_size] = k[b]
+        kp[page, pos % page_size] = rope(k[b][None], [pos], theta)[0] if rotate_k else k[b]
         vp[page, pos % page_size] = v[b]
     return q, kp, vp
 
