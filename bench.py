@@ -356,7 +356,7 @@ def config_entry(w, *, world, step_ms, attn_ms, peaks, peak_src, cpu_base, clock
 
 def build_line(*, world, K, W, only, do_p, do_d, wp, wd, value_tflops, pre_mean, attn_mean, dec_mean, split_mean,
                total_rows, page, peaks, peak_src, cpu_base, e2e_pre, e2e_dec, pre_io, dec_io, qkv_line, clocks,
-               t_wall, configs=None, dec_alone=(float("nan"), float("nan"))):
+               t_wall, configs=None, dec_alone=(float("nan"), float("nan")), dec_rot=(float("nan"), float("nan"))):
     """The JSON line of the `ours` arm from the measured numbers (no device work, so the CPU tests cover it).
     Times in ms; pre_io / dec_io = (host->device, device->host) bytes of one end-to-end prefill / decode
     step; a leg that did not run carries NaN, which clean() turns into null."""
@@ -401,6 +401,7 @@ def build_line(*, world, K, W, only, do_p, do_d, wp, wd, value_tflops, pre_mean,
         "gpu_launches": (2 * do_p + 3 * do_d) * 2 * K + (6 * K if qkv_line else 0)
                         + 2 * 2 * K * sum(1 for n in (configs or {}) if n != wp.name)
                         + (3 * 2 * K if dec_alone[0] == dec_alone[0] else 0)
+                        + ((2 + 3) * K if dec_rot[0] == dec_rot[0] else 0)
                         + ((2 + 3) * K if e2e_pre == e2e_pre else 0),
         "qkv": qkv_line,
         "clocks": clocks,
@@ -421,6 +422,12 @@ def build_line(*, world, K, W, only, do_p, do_d, wp, wd, value_tflops, pre_mean,
                       "split_frac": allb / (dec_alone[1] * 1e-3) / 1e9 / peaks["hbm_gbs"],
                       "note": "the same decode in steps of its own (L2 flushed before each), timed before the "
                               "prefill legs, on a GPU not yet warm"},
+            "rotated_cache": {"ms_per_step": dec_rot[0], "value": world * allb / (dec_rot[0] * 1e-3) / 1e9,
+                              "unit": "GB/s", "split_ms_per_launch": dec_rot[1],
+                              "split_frac": allb / (dec_rot[1] * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                              "note": "the same decode over a cache that keeps its keys after RoPE "
+                                      "(gqa_set_decode_cache_rotated(1)): only the query is rotated; each step "
+                                      "follows the prefill as in the headline step (events around the decode)"},
             "e2e": {"value": world * allb / (e2e_dec * 1e-3) / 1e9, "unit": "GB/s",
                     "h2d_bytes_per_step": dec_io[0], "d2h_bytes_per_step": dec_io[1],
                     "note": "the KV cache is resident device state; the step's inputs are q, the lengths"
@@ -582,6 +589,33 @@ def run_ours(args):
     dec_mean = reduce_max(sum(dec_ms) / K, dev)
     attn_mean = sum(attn_ms) / K
     split_mean = sum(split_ms) / K
+
+    # ---- the same decode over a cache that keeps its keys after RoPE (gqa_set_decode_cache_rotated): the
+    # decode rotates only the query.  Random keys serve as rotated keys as well as raw ones, so the same
+    # cache is used.  Each step follows the prefill, as the headline step's decode half does.
+    dec_rot_ms = split_rot_ms = float("nan")
+    if do_d and do_p:
+        rv = [[ev() for _ in range(4)] for _ in range(K)]
+        torch.cuda.synchronize()
+        barrier()
+        G.set_decode_cache_rotated(True)
+        try:
+            for i in range(K):
+                flush.zero_()
+                G.prefill(q, k, v, theta=wp.theta, out=out)
+                rv[i][0].record()
+                G.set_timing_events(rv[i][1], rv[i][2])
+                dec_call(qd, s, table)
+                G.set_timing_events(None, None)
+                rv[i][3].record()
+            torch.cuda.synchronize()
+        finally:
+            G.set_decode_cache_rotated(False)
+        barrier()
+        if G.last_error() != 0:
+            raise RuntimeError("device error in the rotated-cache decode leg")
+        dec_rot_ms = reduce_max(sum(e[0].elapsed_time(e[3]) for e in rv) / K, dev)
+        split_rot_ms = sum(e[1].elapsed_time(e[2]) for e in rv) / K
 
     # ---- end to end through the public API: every step copies its inputs in from pinned host memory, runs
     # the call and copies its result out to pinned host memory.  The prefill steps are pipelined as a
@@ -748,7 +782,7 @@ def run_ours(args):
             pre_io=(sum(x.numel() * x.element_size() for x in (q, k, v)), out.numel() * out.element_size()),
             dec_io=(qd.numel() * 2 + s.numel() * 4 + (table.numel() * 4 if page else 0), outd.numel() * 2),
             qkv_line=qkv_line, clocks=sampler.summary(), t_wall=t_wall, configs=configs,
-            dec_alone=(dec_alone_ms, split_alone_ms))
+            dec_alone=(dec_alone_ms, split_alone_ms), dec_rot=(dec_rot_ms, split_rot_ms))
     if torch.distributed.is_initialized():
         barrier()
         torch.distributed.destroy_process_group()

@@ -47,10 +47,12 @@ def load() -> ctypes.CDLL:
     lib.gqa_decode_paged.restype = i
     lib.gqa_qkv_rope.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f]
     lib.gqa_qkv_rope.restype = i
-    lib.gqa_qkv_append.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i]
+    lib.gqa_qkv_append.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, f]
     lib.gqa_qkv_append.restype = i
     lib.gqa_set_decode_self_in_cache.argtypes = [i]
     lib.gqa_set_decode_self_in_cache.restype = i
+    lib.gqa_set_decode_cache_rotated.argtypes = [i]
+    lib.gqa_set_decode_cache_rotated.restype = i
     lib.gqa_prefill_rotated.argtypes = [vp, vp, vp, vp, i, i, i, i, i]
     lib.gqa_prefill_rotated.restype = i
     lib.gqa_out_proj.argtypes = [vp, vp, vp, vp, i, i, i]
@@ -212,10 +214,11 @@ def qkv_rope(x: torch.Tensor, w_qkv: torch.Tensor, b_qkv: torch.Tensor | None, h
 
 def qkv_append(x: torch.Tensor, w_qkv: torch.Tensor, b_qkv: torch.Tensor | None, h_q: int, h_kv: int,
                seqlens: torch.Tensor, kpages: torch.Tensor, vpages: torch.Tensor, block_table: torch.Tensor,
-               q: torch.Tensor | None = None) -> torch.Tensor:
+               q: torch.Tensor | None = None, theta: float = 1.0e6) -> torch.Tensor:
     """One decode step's projection and cache append.  x [B, d_model] (the new token of each sequence);
     w_qkv, b_qkv as for qkv_rope; seqlens int32 [B] (device): each new token's position (the cache length
-    before the append).  Writes the tokens' K (un-rotated) and V into kpages / vpages [num_pages, page_size,
+    before the append).  Writes the tokens' K (un-rotated, or rotated at its position with base `theta`
+    while set_decode_cache_rotated(True) is in effect) and V into kpages / vpages [num_pages, page_size,
     h_kv, d] at those positions through block_table int32 [B, max_pages]; returns q [B, h_q, d] (un-rotated)."""
     if x.dim() != 2 or w_qkv.dim() != 2 or kpages.dim() != 4:
         raise ValueError("x must be [B, d_model], w_qkv [(h_q + 2 h_kv) d, d_model], kpages [P, page, h_kv, d]")
@@ -242,7 +245,7 @@ def qkv_append(x: torch.Tensor, w_qkv: torch.Tensor, b_qkv: torch.Tensor | None,
         _stream(x.device)
         rc = load().gqa_qkv_append(_ptr(x), _ptr(w_qkv), _ptr(b_qkv), _ptr(seqlens), _ptr(q), _ptr(kpages),
                                    _ptr(vpages), _ptr(block_table), B, dm, h_q, h_kv, d, page_size, num_pages,
-                                   block_table.shape[1])
+                                   block_table.shape[1], float(theta))
     if rc != GQA_OK:
         raise GQAError(rc, "gqa_qkv_append")
     return q
@@ -254,6 +257,15 @@ def set_decode_self_in_cache(on: bool) -> None:
     rc = load().gqa_set_decode_self_in_cache(1 if on else 0)
     if rc != GQA_OK:
         raise GQAError(rc, "gqa_set_decode_self_in_cache")
+
+
+def set_decode_cache_rotated(on: bool) -> None:
+    """Later decode / append / qkv_rope calls: False (default) -- the K cache holds raw keys, rotated by the
+    decode on load; True -- it holds keys already rotated at their positions (qkv_append and qkv_rope's k
+    output write them so), and the decode rotates only the query."""
+    rc = load().gqa_set_decode_cache_rotated(1 if on else 0)
+    if rc != GQA_OK:
+        raise GQAError(rc, "gqa_set_decode_cache_rotated")
 
 
 def prefill_rotated(qr: torch.Tensor, kr: torch.Tensor, v: torch.Tensor, out: torch.Tensor | None = None):

@@ -197,7 +197,9 @@ __device__ __forceinline__ void rot_step(uint64_t& C, uint64_t& S, uint64_t Cr, 
 }
 
 // PAGED: cache rows are read through the block table p.bt (gqa_decode_paged); otherwise packed.
-template <int D, bool PAGED>
+// KROT: the cached keys are already rotated at their positions (a cache that keeps keys after RoPE), so
+// they go to the dot product as loaded; otherwise each key is rotated on load at its row index.
+template <int D, bool PAGED, bool KROT>
 __global__ void __launch_bounds__(WARPS * 32, CTAS_PER_SM) split_kernel(const Params p) {
     using C = Cfg<D>;
     constexpr int H = D / 2;
@@ -378,7 +380,7 @@ __global__ void __launch_bounds__(WARPS * 32, CTAS_PER_SM) split_kernel(const Pa
             const int nvalid = static_cast<int>(seg_end - cur.r < ROWS ? seg_end - cur.r : ROWS);
             const int64_t jb = cur.r - seq0;   // position of the block's first row
 
-            if (since_anchor >= REANCHOR) {
+            if (!KROT && since_anchor >= REANCHOR) {
 #pragma unroll
                 for (int fp = 0; fp < C::NP; ++fp) {
                     const int di = 16 * (fp >> 1) + 2 * tq + 8 * (fp & 1);
@@ -403,7 +405,7 @@ __global__ void __launch_bounds__(WARPS * 32, CTAS_PER_SM) split_kernel(const Pa
                 ldsm_x4(krow + 16 * ks * 2, a[0], a[1], a[2], a[3]);
                 ldsm_x4(krow + 16 * (ks + C::HALF_KS) * 2, a2[0], a2[1], a2[2], a2[3]);
 #pragma unroll
-                for (int hf = 0; hf < 2; ++hf) {   // dims 16ks + 2tq + 8*hf + {0, 1}
+                for (int hf = 0; hf < (KROT ? 0 : 2); ++hf) {   // dims 16ks + 2tq + 8*hf + {0, 1}
                     const int fp = 2 * ks + hf;
                     const float4 r8 = rot8[(16 * ks + 2 * tq + 8 * hf) >> 1];
                     const uint64_t Cr = f2_pack(r8.x, r8.y), Sr = f2_pack(r8.z, r8.w);

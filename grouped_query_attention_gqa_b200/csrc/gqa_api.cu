@@ -78,6 +78,11 @@ cudaEvent_t g_ev_start = nullptr, g_ev_stop = nullptr;   // optional timing of t
 // 1 = at seqlens[b] - 1, the cache's last row being the query's own.
 int g_self_in_cache = 0;
 
+// Whether the decode caches keep their keys after RoPE (gqa_set_decode_cache_rotated): 0 = raw keys, rotated
+// on load by the decode; 1 = keys already rotated at their positions (with the YaRN temperature), written so
+// by gqa_qkv_rope's k output and by gqa_qkv_append.
+int g_cache_rotated = 0;
+
 // YaRN scaling of RoPE for every later call (gqa_set_rope_scaling); factor 1 = plain RoPE.
 float g_rope_factor = 1.0f;
 int g_rope_orig = 0;
@@ -542,6 +547,7 @@ int launch_qkv(DeviceState* st, const void* x, const void* w, const void* bias, 
     Params p = {};
     p.bias = static_cast<const __nv_bfloat16*>(bias);
     p.tab = static_cast<const float2*>(st->tab);
+    p.k_rotated = g_cache_rotated;
     p.qr = static_cast<__nv_bfloat16*>(qr);
     p.kr = static_cast<__nv_bfloat16*>(kr);
     p.k = static_cast<__nv_bfloat16*>(k);
@@ -586,7 +592,7 @@ int launch_proj(DeviceState* st, const void* attn, const void* w_o, const void* 
 template <int D>
 int launch_append(DeviceState* st, const void* x, const void* w, const void* bias, const int* seqlens, void* q,
                   void* kpages, void* vpages, const int* bt, int B, int d_model, int h_q, int h_kv, int page_size,
-                  int num_pages, int max_pages) {
+                  int num_pages, int max_pages, float theta) {
     using namespace gqa::qkv;
     const int N = (h_q + 2 * h_kv) * D;
     const long long mtiles = (static_cast<long long>(B) + BM - 1) / BM;
@@ -602,6 +608,9 @@ int launch_append(DeviceState* st, const void* x, const void* w, const void* bia
     p.page_size = page_size;
     p.num_pages = num_pages;
     p.max_pages = max_pages;
+    p.k_rotated = g_cache_rotated;
+    p.rope = rope_spec(theta);
+    p.mscale = rope_mscale();
     p.T = B;
     p.L = 1;
     p.N = N;
@@ -626,7 +635,8 @@ int launch_decode_chain(const gqa::decode::Params& p, const int* seqlens, int64_
     const long long cgrid = static_cast<long long>(p.B) * p.h_kv * p.n_hb;
     if (cgrid > 0x7fffffffLL) return GQA_ERR_DIMS;
     const bool paged = p.bt != nullptr;
-    auto split = paged ? split_kernel<D, true> : split_kernel<D, false>;
+    auto split = paged ? (g_cache_rotated ? split_kernel<D, true, true> : split_kernel<D, true, false>)
+                       : (g_cache_rotated ? split_kernel<D, false, true> : split_kernel<D, false, false>);
     if (cudaFuncSetAttribute(split, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
         return GQA_ERR_LAUNCH;
     const bool timed = marks && g_ev_start && g_ev_stop;
@@ -691,7 +701,8 @@ int launch_decode(DeviceState* st, const void* q, const void* kc, const void* vc
     p.self_in_cache = g_self_in_cache;
     p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
     p.rope = rope_spec(theta);
-    p.scale_log2 *= rope_mscale() * rope_mscale();   // YaRN temperature (1 without scaling)
+    // YaRN temperature on q and on each key (1 without scaling); a rotated cache's keys already carry theirs.
+    p.scale_log2 *= rope_mscale() * (g_cache_rotated ? 1.0f : rope_mscale());
     p.err = st->err;
 
     return launch_decode_chain<D>(p, seqlens, static_cast<int64_t*>(st->dws), G * groups, true);
@@ -758,7 +769,8 @@ int launch_decode_fixed_scratch(DeviceState* st, const void* q, const void* kc, 
     p.self_in_cache = g_self_in_cache;
     p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
     p.rope = rope_spec(theta);
-    p.scale_log2 *= rope_mscale() * rope_mscale();   // YaRN temperature (1 without scaling)
+    // YaRN temperature on q and on each key (1 without scaling); a rotated cache's keys already carry theirs.
+    p.scale_log2 *= rope_mscale() * (g_cache_rotated ? 1.0f : rope_mscale());
     p.err = st->err;
 
     return launch_decode_chain<D>(p, seqlens, static_cast<int64_t*>(st->fixed_scratch), G * groups, false);
@@ -768,7 +780,7 @@ int launch_decode_fixed_scratch(DeviceState* st, const void* q, const void* kc, 
 
 extern "C" {
 
-int gqa_abi_version(void) { return 1; }
+int gqa_abi_version(void) { return 2; }
 
 const char* gqa_strerror(int code) {
     switch (code) {
@@ -892,12 +904,12 @@ int gqa_qkv_rope(const void* x, const void* w_qkv, const void* b_qkv, void* qr, 
 
 int gqa_qkv_append(const void* x, const void* w_qkv, const void* b_qkv, const int* seqlens, void* q, void* kpages,
                    void* vpages, const int* block_table, int B, int d_model, int h_q, int h_kv, int d, int page_size,
-                   int num_pages, int max_pages_per_seq) {
+                   int num_pages, int max_pages_per_seq, float theta) {
     if (B < 0 || d_model <= 0 || d_model % 8 != 0 || page_size <= 0 || num_pages <= 0 || max_pages_per_seq <= 0)
         return GQA_ERR_DIMS;
     if (static_cast<long long>(num_pages) * page_size > (1LL << 40)) return GQA_ERR_DIMS;
     if (static_cast<long long>(B) * max_pages_per_seq > 0x7fffffffLL) return GQA_ERR_DIMS;
-    int rc = check_common(h_q, h_kv, d, 1.0f);
+    int rc = check_common(h_q, h_kv, d, theta);
     if (rc != GQA_OK) return rc;
     if (B == 0) return GQA_OK;
     if (!x || !w_qkv || !seqlens || !q || !kpages || !vpages || !block_table) return GQA_ERR_NULL;
@@ -908,14 +920,20 @@ int gqa_qkv_append(const void* x, const void* w_qkv, const void* b_qkv, const in
     DeviceState* st = device_state(&rc);
     if (!st) return rc;
     return d == 64 ? launch_append<64>(st, x, w_qkv, b_qkv, seqlens, q, kpages, vpages, block_table, B, d_model, h_q,
-                                       h_kv, page_size, num_pages, max_pages_per_seq)
+                                       h_kv, page_size, num_pages, max_pages_per_seq, theta)
                    : launch_append<128>(st, x, w_qkv, b_qkv, seqlens, q, kpages, vpages, block_table, B, d_model,
-                                        h_q, h_kv, page_size, num_pages, max_pages_per_seq);
+                                        h_q, h_kv, page_size, num_pages, max_pages_per_seq, theta);
 }
 
 int gqa_set_decode_self_in_cache(int on) {
     if (on != 0 && on != 1) return GQA_ERR_DIMS;
     g_self_in_cache = on;
+    return GQA_OK;
+}
+
+int gqa_set_decode_cache_rotated(int on) {
+    if (on != 0 && on != 1) return GQA_ERR_DIMS;
+    g_cache_rotated = on;
     return GQA_OK;
 }
 

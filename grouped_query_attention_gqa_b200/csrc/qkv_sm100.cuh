@@ -71,6 +71,11 @@ struct Params {
     const int* seqlens;
     const int* bt;
     int page_size, max_pages, num_pages;
+    // The caches keep their keys after RoPE: qkv's k output and the append's key rows are written rotated
+    // (the append at position seqlens[t], with `rope` and the YaRN temperature `mscale`).
+    int k_rotated;
+    RopeSpec rope;
+    float mscale;
     int T, L, N, h_q, h_kv;
     int n_ntiles, n_tiles, kblocks;
     // Work units: tiles 0 .. n_main-1 whole (BN columns); each later tile split into tail_split units of
@@ -216,8 +221,9 @@ __device__ __forceinline__ void store_head(const Params& p, float (&y)[D], int n
         store_rows<D>(stage, row_of(p.qr, (static_cast<int64_t>(b) * p.h_q + head) * p.L + pos), y, lane);
     } else if (head < p.h_q + p.h_kv) {
         const int u = head - p.h_q;
+        if (p.k_rotated) rotate(y);   // the cache rows keep the key after RoPE
         store_rows<D>(stage, row_of(p.k, (static_cast<int64_t>(b) * p.L + pos) * p.h_kv + u), y, lane);
-        rotate(y);
+        if (!p.k_rotated) rotate(y);
         store_rows<D>(stage, row_of(p.kr, (static_cast<int64_t>(b) * p.h_kv + u) * p.L + pos), y, lane);
     } else {
         const int u = head - p.h_q - p.h_kv;
@@ -251,9 +257,10 @@ __device__ __forceinline__ void store_resid(const Params& p, float (&y)[W], int 
 // The decode-step append's epilogue: one head of one token row per lane, + bias, stored un-rotated (the
 // decode rotates q and every cached key at its position): a query head to its q row, a key or value head
 // to the token's page slot (kv_row: the slot's row of h_kv heads in the key or value pages, nullptr when
-// the row is past the end or its table entry is invalid).
+// the row is past the end or its table entry is invalid).  Where the caches keep keys after RoPE
+// (p.k_rotated), a key head is rotated at the token's position `at` first.
 template <int D>
-__device__ __forceinline__ void store_append(const Params& p, float (&y)[D], int n0, int t, bool valid,
+__device__ __forceinline__ void store_append(const Params& p, float (&y)[D], int n0, int t, int at, bool valid,
                                              __nv_bfloat16* k_row, __nv_bfloat16* v_row, uint8_t* stage, int lane) {
     if (p.bias) {
         const uint4* bb = reinterpret_cast<const uint4*>(p.bias + n0);
@@ -269,6 +276,17 @@ __device__ __forceinline__ void store_append(const Params& p, float (&y)[D], int
         }
     }
     const int head = n0 / D;
+    if (p.k_rotated && head >= p.h_q && head < p.h_q + p.h_kv && k_row) {
+#pragma unroll
+        for (int i = 0; i < D / 2; ++i) {
+            float c, s;
+            rope_cossin(static_cast<double>(at), rope_freq(i, D, p.rope), c, s);
+            float xr, yr;
+            rope_rotate(y[i], y[i + D / 2], c * p.mscale, s * p.mscale, xr, yr);
+            y[i] = xr;
+            y[i + D / 2] = yr;
+        }
+    }
     __nv_bfloat16* dst;
     if (head < p.h_q) dst = valid ? p.qr + (static_cast<int64_t>(t) * p.h_q + head) * D : nullptr;
     else if (head < p.h_q + p.h_kv) dst = k_row ? k_row + static_cast<int64_t>(head - p.h_q) * D : nullptr;
@@ -446,8 +464,9 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtenso
             const int b = valid ? t / p.L : 0, pos = valid ? t % p.L : 0;
             // kAppend: this row's page slot (rows of all h_kv heads) in the key and value pages
             __nv_bfloat16 *k_row = nullptr, *v_row = nullptr;
+            int at = 0;
             if (EPI == kAppend && valid) {
-                const int at = __ldg(p.seqlens + t);
+                at = __ldg(p.seqlens + t);
                 const int pi = at >= 0 ? at / p.page_size : -1;
                 const int page = (pi >= 0 && pi < p.max_pages) ? __ldg(p.bt + static_cast<int64_t>(t) * p.max_pages + pi) : -1;
                 if (page >= 0 && page < p.num_pages) {
@@ -481,7 +500,7 @@ __device__ __forceinline__ void gemm_body(const CUtensorMap& tm_x, const CUtenso
                                   *reinterpret_cast<uint32_t(*)[32]>(acc + 32 * c));
                     tmem_wait_ld();
                     if (EPI == kQKV) store_head<D>(p, acc, n0, b, pos, valid, stage, lane);
-                    else if (EPI == kAppend) store_append<D>(p, acc, n0, t, valid, k_row, v_row, stage, lane);
+                    else if (EPI == kAppend) store_append<D>(p, acc, n0, t, at, valid, k_row, v_row, stage, lane);
                     else store_resid<128>(p, *reinterpret_cast<float(*)[128]>(acc), n0, t, valid, stage, lane);
                 }
             }

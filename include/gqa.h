@@ -160,6 +160,7 @@ GQA_API int gqa_decode_paged(const void* q, const void* kpages, const void* vpag
  * Outputs (bf16, caller-owned): with Y = x w_qkv^T + b_qkv split into heads, at positions 0 .. L-1,
  *   qr [B, h_q, L, d]   rotated Q, head-major      kr [B, h_kv, L, d]   rotated K, head-major
  *   k  [B, L, h_kv, d]  un-rotated K, token-major  v  [B, L, h_kv, d]   V, token-major
+ *   (k holds the rotated K instead while gqa_set_decode_cache_rotated(1) is in effect)
  * k and v are exactly the packed cache rows of gqa_decode for B sequences of L rows stored back to back,
  * so pointing them into a cache appends the sequences; qr, kr and v are the inputs of
  * gqa_prefill_rotated.  Each output element is the fp32 accumulation rounded to bf16 once.
@@ -182,9 +183,12 @@ GQA_API int gqa_qkv_rope(const void* x, const void* w_qkv, const void* b_qkv, vo
  *   q            [B, h_q, d]   out: the new tokens' queries, un-rotated (the decode entry points rotate the
  *                query at its position)
  *   kpages, vpages [num_pages, page_size, h_kv, d]  the paged cache of gqa_decode_paged: the token's K
- *                (un-rotated, like every cache row) and V are written to slot p_b % page_size of page
+ *                (un-rotated, like every cache row; rotated at p_b when the caches keep keys after RoPE,
+ *                see gqa_set_decode_cache_rotated) and V are written to slot p_b % page_size of page
  *                block_table[b][p_b / page_size]; nothing else in the pages is touched
  *   block_table  [B, max_pages_per_seq] int32, DEVICE memory
+ *   theta        the RoPE base of that key rotation (used only when the caches keep rotated keys; must be
+ *                finite and > 0 in any case, else GQA_ERR_THETA)
  * Each written element is the fp32 accumulation (plus the bias) rounded once to bf16.  A decode loop is
  * then: gqa_qkv_append, then gqa_decode_paged with seqlens[b] + 1 and gqa_set_decode_self_in_cache(1) (the
  * new token attends to itself and to every earlier position), then grow seqlens.  A position outside the
@@ -194,7 +198,7 @@ GQA_API int gqa_qkv_rope(const void* x, const void* w_qkv, const void* b_qkv, vo
  */
 GQA_API int gqa_qkv_append(const void* x, const void* w_qkv, const void* b_qkv, const int* seqlens, void* q,
                            void* kpages, void* vpages, const int* block_table, int B, int d_model, int h_q,
-                           int h_kv, int d, int page_size, int num_pages, int max_pages_per_seq);
+                           int h_kv, int d, int page_size, int num_pages, int max_pages_per_seq, float theta);
 
 /*
  * gqa_set_decode_self_in_cache -- where the query of every later gqa_decode, gqa_decode_paged and
@@ -205,6 +209,19 @@ GQA_API int gqa_qkv_append(const void* x, const void* w_qkv, const void* b_qkv, 
  * seqlens[b] rows, itself included.  Process-global, like the stream.  Returns GQA_ERR_DIMS for other values.
  */
 GQA_API int gqa_set_decode_self_in_cache(int on);
+
+/*
+ * gqa_set_decode_cache_rotated -- what the K cache holds for every later gqa_decode, gqa_decode_paged,
+ * gqa_decode_noalloc and gqa_qkv_append call, and what gqa_qkv_rope writes to its k output.  0 (the
+ * default): raw keys, as projected; the decode rotates each cached key at its row index on load (page
+ * "Qwen2 architecture introduction", §4.1.3: RoPE acts on Q and K before the dot product).  1: keys kept
+ * after RoPE, each already rotated at its own position (with the YaRN temperature when scaling is on), as
+ * a serving cache keeps them; the decode uses them as loaded and rotates only the query, gqa_qkv_append
+ * writes the new key rotated at its position, and gqa_qkv_rope's k output holds the rotated keys
+ * (token-major; kr is unchanged).  The scores are the same either way; the rotated cache saves the decode
+ * the per-key rotation.  Process-global, like the stream.  Returns GQA_ERR_DIMS for other values.
+ */
+GQA_API int gqa_set_decode_cache_rotated(int on);
 
 /*
  * gqa_prefill_rotated -- the causal attention of gqa_prefill on inputs that are already rotated (page

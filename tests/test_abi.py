@@ -32,7 +32,8 @@ def codes():
 def test_header_declares_the_entry_points():
     names = set(declared())
     for n in ["gqa_prefill", "gqa_decode", "gqa_decode_paged", "gqa_qkv_rope", "gqa_prefill_rotated",
-              "gqa_out_proj", "gqa_qkv_append", "gqa_set_decode_self_in_cache", "gqa_set_stream", "gqa_last_error",
+              "gqa_out_proj", "gqa_qkv_append", "gqa_set_decode_self_in_cache", "gqa_set_decode_cache_rotated",
+              "gqa_set_stream", "gqa_last_error",
               "gqa_release",
               "gqa_strerror", "gqa_abi_version", "gqa_set_timing_events"]:
         assert n in names
@@ -44,7 +45,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_version_and_strerror(lib):
-    assert lib.gqa_abi_version() == 1
+    assert lib.gqa_abi_version() == 2
     c = codes()
     for k, v in c.items():
         if k.startswith("GQA_ERR_"):
@@ -173,8 +174,8 @@ def test_set_stream_accepts_null(lib):
 
 
 def append_args(x=P16, w=P16, b=None, s=P16, q=P16, kp=P16, vp=P16, bt=P16, B=2, dm=256, h_q=28, h_kv=4, d=128,
-                page=16, npages=8, maxp=4):
-    return (x, w, b, s, q, kp, vp, bt, B, dm, h_q, h_kv, d, page, npages, maxp)
+                page=16, npages=8, maxp=4, theta=1.0e6):
+    return (x, w, b, s, q, kp, vp, bt, B, dm, h_q, h_kv, d, page, npages, maxp, ctypes.c_float(theta))
 
 
 @pytest.mark.parametrize("args,code", [
@@ -187,6 +188,8 @@ def append_args(x=P16, w=P16, b=None, s=P16, q=P16, kp=P16, vp=P16, bt=P16, B=2,
     (append_args(npages=1 << 30, page=1 << 12), "GQA_ERR_DIMS"),      # storage rows beyond 2^40
     (append_args(h_kv=3), "GQA_ERR_DIMS"),
     (append_args(d=96), "GQA_ERR_HEAD_DIM"),
+    (append_args(theta=0.0), "GQA_ERR_THETA"),
+    (append_args(theta=float("nan")), "GQA_ERR_THETA"),
     (append_args(x=None), "GQA_ERR_NULL"),
     (append_args(s=None), "GQA_ERR_NULL"),
     (append_args(bt=None), "GQA_ERR_NULL"),
@@ -203,3 +206,9 @@ def test_qkv_append_validation(lib, args, code):
 def test_set_decode_self_in_cache_validation(lib, on, code):
     assert lib.gqa_set_decode_self_in_cache(on) == codes()[code]
     lib.gqa_set_decode_self_in_cache(0)
+
+
+@pytest.mark.parametrize("on,code", [(0, "GQA_OK"), (1, "GQA_OK"), (2, "GQA_ERR_DIMS"), (-1, "GQA_ERR_DIMS")])
+def test_set_decode_cache_rotated_validation(lib, on, code):
+    assert lib.gqa_set_decode_cache_rotated(on) == codes()[code]
+    lib.gqa_set_decode_cache_rotated(0)

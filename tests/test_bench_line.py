@@ -16,7 +16,7 @@ CONTRACT = ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step
             "impl")
 
 
-def line_for(only, world=1, page=None, qkv=None, configs=None, dec_alone=(NAN, NAN)):
+def line_for(only, world=1, page=None, qkv=None, configs=None, dec_alone=(NAN, NAN), dec_rot=(NAN, NAN)):
     do_p, do_d = only in (None, "prefill"), only in (None, "decode")
     wp, wd = gi.BY_NAME[bench.PREFILL_WORKLOAD], gi.BY_NAME[bench.DECODE_WORKLOAD]
     fl = bench.prefill_flops(wp)
@@ -30,7 +30,7 @@ def line_for(only, world=1, page=None, qkv=None, configs=None, dec_alone=(NAN, N
         cpu_base={"value": 0.03, "unit": "TFLOP/s", "cores": 16, "kind": "oracle", "sample": "s"} if do_p else None,
         e2e_pre=1.3 if do_p else NAN, e2e_dec=0.4 if do_d else NAN, pre_io=(37748736, 29360128),
         dec_io=(459008, 458752), qkv_line=qkv, clocks={"sm_mhz": 1965, "sm_max_mhz": 1965, "reasons": []},
-        t_wall=0.05, configs=configs, dec_alone=dec_alone)
+        t_wall=0.05, configs=configs, dec_alone=dec_alone, dec_rot=dec_rot)
     text = json.dumps(bench.clean(line), allow_nan=False)   # strict JSON: no NaN or inf survives
     return json.loads(text)
 
@@ -129,3 +129,14 @@ def test_peak_is_sustained_only_for_long_power_capped_runs():
     assert r["peak"] == PEAKS["bf16_tflops_sustained"] and math.isclose(r["frac"], ach / r["peak"])
     assert math.isclose(r["frac_of_burst"], ach / PEAKS["bf16_tflops"])
     assert "sustained" in r["peak_source"]
+
+
+def test_rotated_cache_decode_beside_the_in_step_decode():
+    d = line_for(None, dec_rot=(0.33, 0.315))
+    r = d["decode"]["rotated_cache"]
+    allb = bench.decode_bytes(954557, gi.BY_NAME[bench.DECODE_WORKLOAD])
+    assert abs(r["split_frac"] - allb / (0.315e-3) / 1e9 / PEAKS["hbm_gbs"]) < 1e-9
+    assert abs(r["value"] - allb / (0.33e-3) / 1e9) < 1e-6
+    # its K steps of prefill + decode count among the line's launches
+    assert d["gpu_launches"] == line_for(None)["gpu_launches"] + (2 + 3) * 30
+    assert line_for(None)["decode"]["rotated_cache"]["value"] is None
