@@ -356,7 +356,8 @@ def config_entry(w, *, world, step_ms, attn_ms, peaks, peak_src, cpu_base, clock
 
 def build_line(*, world, K, W, only, do_p, do_d, wp, wd, value_tflops, pre_mean, attn_mean, dec_mean, split_mean,
                total_rows, page, peaks, peak_src, cpu_base, e2e_pre, e2e_dec, pre_io, dec_io, qkv_line, clocks,
-               t_wall, configs=None, dec_alone=(float("nan"), float("nan")), dec_rot=(float("nan"), float("nan"))):
+               t_wall, configs=None, dec_alone=(float("nan"), float("nan")), dec_rot=(float("nan"), float("nan")),
+               k_cache="raw"):
     """The JSON line of the `ours` arm from the measured numbers (no device work, so the CPU tests cover it).
     Times in ms; pre_io / dec_io = (host->device, device->host) bytes of one end-to-end prefill / decode
     step; a leg that did not run carries NaN, which clean() turns into null."""
@@ -409,13 +410,16 @@ def build_line(*, world, K, W, only, do_p, do_d, wp, wd, value_tflops, pre_mean,
             "workload": wd.desc, "total_cache_rows": total_rows,
             "layout": f"paged: {page} rows per page, pages scattered in a seeded random order" if page
                       else "packed",
+            "k_cache": "keys kept after RoPE (gqa_set_decode_cache_rotated(1)): only the query is rotated"
+                       if k_cache == "rotated" else "raw keys, each rotated on load at its position",
             "value": world * allb / (dec_mean * 1e-3) / 1e9, "unit": "GB/s",
             "kv_gbs": world * kvb / (dec_mean * 1e-3) / 1e9,
             "ms_per_step": dec_mean,
             "roofline": {"kernel": "split_kernel (decode)", "bound": "hbm", "achieved": achieved_b,
                          "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": achieved_b / peaks["hbm_gbs"],
                          "peak_source": f"{peak_src} HBM copy",
-                         "traffic": profile_traffic("split_kernel", DECODE_WORKLOAD + (f"-paged{page}" if page else "")),
+                         "traffic": profile_traffic("split_kernel", DECODE_WORKLOAD + (f"-paged{page}" if page else "")
+                                                    + ("-rotated" if k_cache == "rotated" else "")),
                          "algorithmic_bytes_per_launch": allb, "ms_per_launch": split_mean},
             "alone": {"ms_per_step": dec_alone[0], "value": world * allb / (dec_alone[0] * 1e-3) / 1e9, "unit": "GB/s",
                       "split_ms_per_launch": dec_alone[1],
@@ -425,6 +429,8 @@ def build_line(*, world, K, W, only, do_p, do_d, wp, wd, value_tflops, pre_mean,
             "rotated_cache": {"ms_per_step": dec_rot[0], "value": world * allb / (dec_rot[0] * 1e-3) / 1e9,
                               "unit": "GB/s", "split_ms_per_launch": dec_rot[1],
                               "split_frac": allb / (dec_rot[1] * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                              "traffic": profile_traffic("split_kernel", DECODE_WORKLOAD
+                                                         + (f"-paged{page}" if page else "") + "-rotated"),
                               "note": "the same decode over a cache that keeps its keys after RoPE "
                                       "(gqa_set_decode_cache_rotated(1)): only the query is rotated; each step "
                                       "follows the prefill as in the headline step (events around the decode)"},
@@ -471,6 +477,10 @@ def run_ours(args):
         q, k, v = (torch.empty(1, 1, 1, 8, dtype=torch.bfloat16, device=dev) for _ in range(3))
     out = torch.empty_like(q)
     page = args.decode_page_size
+    # --decode-cache rotated: every decode of the run reads a cache that keeps its keys after RoPE (random
+    # keys serve as rotated keys as well as raw ones, so the same cache is used)
+    rotated_run = args.decode_cache == "rotated"
+    G.set_decode_cache_rotated(rotated_run)
     table = None
     if do_d and page:   # the same logical cache, scattered over pages of `page` rows
         s, qd, kc, vc, table, _, _, _ = gi.decode_paged_inputs(wd, page, device=str(dev))
@@ -594,7 +604,7 @@ def run_ours(args):
     # decode rotates only the query.  Random keys serve as rotated keys as well as raw ones, so the same
     # cache is used.  Each step follows the prefill, as the headline step's decode half does.
     dec_rot_ms = split_rot_ms = float("nan")
-    if do_d and do_p:
+    if do_d and do_p and not rotated_run:
         rv = [[ev() for _ in range(4)] for _ in range(K)]
         torch.cuda.synchronize()
         barrier()
@@ -782,7 +792,7 @@ def run_ours(args):
             pre_io=(sum(x.numel() * x.element_size() for x in (q, k, v)), out.numel() * out.element_size()),
             dec_io=(qd.numel() * 2 + s.numel() * 4 + (table.numel() * 4 if page else 0), outd.numel() * 2),
             qkv_line=qkv_line, clocks=sampler.summary(), t_wall=t_wall, configs=configs,
-            dec_alone=(dec_alone_ms, split_alone_ms), dec_rot=(dec_rot_ms, split_rot_ms))
+            dec_alone=(dec_alone_ms, split_alone_ms), dec_rot=(dec_rot_ms, split_rot_ms), k_cache=args.decode_cache)
     if torch.distributed.is_initialized():
         barrier()
         torch.distributed.destroy_process_group()
@@ -808,6 +818,9 @@ def main(argv=None):
                     help="comma list of further prefill workloads timed before the headline and reported under "
                          "`configs` ('none' for none)")
     ap.add_argument("--no-qkv", action="store_true", help="skip the fused QKV projection leg")
+    ap.add_argument("--decode-cache", choices=["raw", "rotated"], default="raw",
+                    help="what the decode's K cache holds: raw keys rotated on load (default), or keys kept after "
+                         "RoPE (gqa_set_decode_cache_rotated)")
     ap.add_argument("--decode-page-size", type=int, default=None,
                     help="decode through gqa_decode_paged, the cache in pages of this many rows")
     ap.add_argument("--decode-batch", type=int, default=None,
