@@ -159,3 +159,31 @@ def test_noalloc_refuses_problems_far_beyond_its_fixed_scratch(lib):
     rc = lib.gqa_decode_noalloc(_p(q), _p(kc), _p(kc), _p(s), _p(out), B, 28, 4, 128, ctypes.c_float(1e6))
     assert rc == GQA_ERR_TOO_LARGE
     assert torch.count_nonzero(out).item() == 0   # nothing was launched
+
+
+def test_noalloc_over_a_cache_that_keeps_keys_after_rope(lib):
+    """With gqa_set_decode_cache_rotated(1) the no-allocation decode reads the keys as already rotated at
+    their positions, like gqa_decode: the two agree bit for bit and match the oracle's k_rotated decode."""
+    dev = torch.device("cuda")
+    w = gi.small("decode", B=5, max_len=2100, h_q=28, h_kv=4, d=128, seed=35)
+    lens = [2100, 1, 640, 17, 1000]
+    s_h, q_h, kc_h, vc_h = gi.decode_inputs(w, seqlens=lens)
+    off = R.packed_offsets(lens)
+    krot_h = torch.from_numpy(np.concatenate([R.rope(R.as_f64(kc_h[off[b]:off[b + 1]]), np.arange(lens[b]), w.theta)
+                                              for b in range(w.B)])).to(torch.bfloat16)
+    s, q, krot, vc = (x.to(dev) for x in (s_h, q_h, krot_h, vc_h))
+    ref = torch.empty_like(q)
+    got = torch.full_like(q, float("nan"))
+    lib.gqa_set_stream(ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    args = (w.B, w.h_q, w.h_kv, w.d, ctypes.c_float(w.theta))
+    assert lib.gqa_set_decode_cache_rotated(1) == 0
+    try:
+        assert lib.gqa_decode(_p(q), _p(krot), _p(vc), _p(s), _p(ref), *args) == 0
+        assert lib.gqa_decode_noalloc(_p(q), _p(krot), _p(vc), _p(s), _p(got), *args) == 0
+        torch.cuda.synchronize()
+    finally:
+        lib.gqa_set_decode_cache_rotated(0)
+    assert lib.gqa_last_error() == 0
+    assert torch.equal(got, ref)
+    oracle = R.decode_ref(q_h, krot_h, vc_h, s_h, w.theta, k_rotated=True)
+    assert_close(got.float().cpu().numpy(), oracle, "gqa_decode_noalloc over a rotated cache vs the oracle")
