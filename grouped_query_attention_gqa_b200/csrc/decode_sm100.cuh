@@ -5,8 +5,7 @@
 // §2.4).  The query of sequence b sits at position p = seqlens[b] and attends to
 // all seqlens[b] cached rows (positions 0 .. p-1).
 //
-// The step is bound by the HBM stream of the cache, so the design is about
-// streaming, not arithmetic:
+// The step streams the whole cache from HBM once, so the design is about streaming:
 //  * plan_kernel   : prefix sums of seqlens -> packed row offsets (one CTA).
 //  * split_kernel  : for each KV group u (and block of <= 8 query heads), the
 //    flattened cache rows [0, N) are cut into P equal slices, one per warp, so
@@ -19,8 +18,12 @@
 //    Each warp owns a 2-stage ring of 16-row blocks filled by 1-D bulk copies
 //    (one row of K or V per lane, padded rows so ldmatrix is conflict-free).
 //    K rows are rotated in registers (RoPE on load) with cos/sin advanced by
-//    an angle-addition recurrence, re-anchored exactly every 64 blocks; the
-//    g <= 8 query heads of the group share every K/V row read.  Scores and PV
+//    an angle-addition recurrence, re-anchored exactly every 64 blocks; that
+//    rotation is most of a block's instructions, enough to make the kernel
+//    follow the SM clock once it drops under the power cap.  Over a cache that
+//    keeps its keys after RoPE (KROT) the rows are used as loaded and the
+//    kernel stays at the HBM stream.  The g <= 8 query heads of the group share
+//    every K/V row read.  Scores and PV
 //    use the warp-level bf16 tensor-core instruction with the key rows as the
 //    M dimension, so the 7 or 8 heads fill the N = 8 dimension.
 //  * combine_kernel: log-sum-exp merge of the pieces of each sequence.

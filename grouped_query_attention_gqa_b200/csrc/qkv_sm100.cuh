@@ -5,6 +5,7 @@
 //   qr [B, h_q,  L, d]  rotated Q, head-major (the attention kernel's Q' layout)
 //   kr [B, h_kv, L, d]  rotated K, head-major (its K' layout)
 //   k  [B, L, h_kv, d]  raw K, token-major: the packed cache rows of the sequences, back to back
+//                       (the rotated K instead for caches that keep keys after RoPE, p.k_rotated)
 //   v  [B, L, h_kv, d]  V, token-major (cache rows; the attention kernel reads V in this layout)
 //
 // qkv_kernel is a persistent tcgen05 GEMM, one CTA per SM, over 128 x 256 output tiles (128 tokens,
