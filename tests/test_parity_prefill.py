@@ -38,6 +38,8 @@ SMALL = [
     (1, 513, 28, 4, 128),
     (3, 200, 16, 4, 128),
     (1, 1000, 4, 1, 64),
+    (1, 300, 32, 2, 128),   # g = 16
+    (2, 257, 6, 2, 64),     # g = 3, a ragged last tile
 ]
 
 
@@ -141,3 +143,27 @@ def test_prefill_full_size_sampled_rows(G, name):
             got = out[b, torch.as_tensor(rows, device=dev), t].float().cpu().numpy()
             ref = R.prefill_rows_ref(q, k, v, w.theta, b, t, rows)
             assert_close(got, ref, f"{name} b={b} t={t}")
+
+
+@pytest.mark.parametrize("B,L,h_q,h_kv,d,expect_grouped", [
+    (2, 4096, 28, 4, 128, False),   # many items per CTA, every plane's K' and V in L2: the round-robin lists
+    (4, 2048, 14, 2, 64, False),    # the same with d = 64
+    (16, 2048, 28, 4, 128, True),   # 64 planes of 1 MB: 64 MB of K' and V, dealt plane group by plane group
+])
+def test_prefill_schedule_paths_sampled_rows(G, B, L, h_q, h_kv, d, expect_grouped):
+    """The attention kernel's other work schedules, checked on sampled rows of the first, a middle and the
+    last batch row and of the first, a middle and the last head."""
+    lists, grouped = G.prefill_schedule(B, L, h_q, h_kv, 148)
+    assert grouped == expect_grouped
+    w = gi.small("prefill", B=B, L=L, h_q=h_q, h_kv=h_kv, d=d, seed=B * 100 + L)
+    q, k, v = gi.prefill_inputs(w)
+    dev = torch.device("cuda")
+    out = G.prefill(q.to(dev), k.to(dev), v.to(dev), theta=w.theta)
+    assert G.last_error() == 0
+    rng = np.random.default_rng(B + L)
+    for b in sorted({0, B // 2, B - 1}):
+        for t in sorted({0, h_q // 2, h_q - 1}):
+            rows = sample_rows(L, rng)
+            got = out[b, torch.as_tensor(rows, device=dev), t].float().cpu().numpy()
+            ref = R.prefill_rows_ref(q, k, v, w.theta, b, t, rows)
+            assert_close(got, ref, f"B={B} L={L} b={b} t={t}")
