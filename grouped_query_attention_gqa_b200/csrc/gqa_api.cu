@@ -225,7 +225,7 @@ int encode_prefill_maps(CUtensorMap* maps, const void* qr, const void* kr, const
 // Per-item overhead of the attention kernel in key tiles, for the schedule below: the start of a pair
 // (its query tiles' loads and first scores) and its epilogue.  Measured: with 0 the packing gives some
 // CTAs many small items and the kernel is 19 % slower than round-robin at L=4096; 2, 4 and 8 are 3 %,
-// 4 % and 2 % faster.
+// 4 % and 2 % faster; against 4, 3 is 4 % slower and 5 the same.
 #ifndef GQA_SCHED_ITEM_COST
 #define GQA_SCHED_ITEM_COST 4
 #endif
