@@ -439,6 +439,9 @@ __global__ void __launch_bounds__(WARPS * 32, CTAS_PER_SM) split_kernel(const Pa
             }
             const float mn0 = fmaxf(m0, bm0), mn1 = fmaxf(m1, bm1);
             const float al0 = ex2(m0 - mn0), al1 = ex2(m1 - mn1);
+            // Once a sequence's running maximum settles it rarely grows: the rescale of O below is then a
+            // multiplication by exactly 1 in every lane, and is skipped (the result is the same bit for bit).
+            const bool grew = __any_sync(0xffffffffu, (mn0 > m0) | (mn1 > m1));
             m0 = mn0;
             m1 = mn1;
             const float p0 = ex2(x0 - m0), p1 = ex2(x1 - m1), p2 = ex2(x2 - m0), p3 = ex2(x3 - m1);
@@ -449,12 +452,17 @@ __global__ void __launch_bounds__(WARPS * 32, CTAS_PER_SM) split_kernel(const Pa
 
             // ---- O^T += V^T P^T  (M = 16 dims per tile, N = 8 heads, K = 16 rows)
             const uint32_t vrow = v_a + ((lane & 7) + 8 * (lane >> 4)) * C::ROWB + 8 * ((lane >> 3) & 1) * 2;
+            if (grew) {
+#pragma unroll
+                for (int mt = 0; mt < C::KS; ++mt) {
+                    o[mt][0] *= al0;
+                    o[mt][1] *= al1;
+                    o[mt][2] *= al0;
+                    o[mt][3] *= al1;
+                }
+            }
 #pragma unroll
             for (int mt = 0; mt < C::KS; ++mt) {
-                o[mt][0] *= al0;
-                o[mt][1] *= al1;
-                o[mt][2] *= al0;
-                o[mt][3] *= al1;
                 uint32_t v0, v1, v2, v3;
                 ldsm_x4_t(vrow + 16 * mt * 2, v0, v1, v2, v3);
                 mma_bf16_16816(o[mt], v0, v1, v2, v3, pb0, pb1);
