@@ -168,3 +168,28 @@ def test_qkv_rope_k_output_holds_the_rotated_keys(G):
     qr0, kr0, k0, v0 = G.qkv_rope(x.to(dev), wq.to(dev), b.to(dev), w.h_q, w.h_kv, theta=w.theta)
     assert torch.equal(kr0, kr) and torch.equal(qr0, qr) and torch.equal(v0, v)
     assert not torch.equal(k0, k)
+
+
+@pytest.mark.parametrize("page", [1, 5])
+def test_rotated_paged_cache_small_pages(G, page):
+    """Pages shorter than a 16-row block (the per-row table lookup of the paged decode) over a rotated
+    cache: bit-identical to the rotated packed decode and within tolerance of the oracle."""
+    w = gi.small("decode", B=4, max_len=700, h_q=28, h_kv=4, d=128, seed=410 + page)
+    lens = [700, 1, 33, 250]
+    s, q, kp, vp, table, npages, kc, vc = gi.decode_paged_inputs(w, page, seqlens=lens)
+    krot = rotate_cache(kc, s.numpy(), w.theta)
+    _, _, store_row = gi.paged_layout(s, page, w.seed + 7919, 3)
+    kp_rot = kp.reshape(-1, w.h_kv, w.d).clone()
+    kp_rot[store_row] = krot
+    kp_rot = kp_rot.reshape(kp.shape)
+    dev = torch.device("cuda")
+    G.set_decode_cache_rotated(True)
+    try:
+        packed = G.decode(q.to(dev), krot.to(dev), vc.to(dev), s.to(dev), theta=w.theta)
+        paged = G.decode_paged(q.to(dev), kp_rot.to(dev), vp.to(dev), table.to(dev), s.to(dev), theta=w.theta)
+    finally:
+        G.set_decode_cache_rotated(False)
+    assert G.last_error() == 0
+    assert torch.equal(paged, packed)
+    ref = R.decode_ref(q, krot, vc, s.numpy(), w.theta, k_rotated=True)
+    assert_close(paged.float().cpu().numpy(), ref, f"rotated cache, {page}-row pages")
