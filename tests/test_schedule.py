@@ -8,6 +8,7 @@ import ctypes
 
 import numpy as np
 import pytest
+from hypothesis import given, settings, strategies as st
 
 import grouped_query_attention_gqa_b200 as G
 from grouped_query_attention_gqa_b200 import _lib
@@ -122,3 +123,30 @@ def test_small_capacity_leaves_arrays_untouched():
     n = lib.gqa_prefill_schedule(1, 4096, 28, 4, 148, starts, items, 4, None)
     assert n == 448
     assert list(starts) == [-7] * 149 and list(items) == [-7] * 4
+
+
+@settings(max_examples=60, deadline=None)
+@given(B=st.integers(1, 6), L=st.integers(1, 9000), h_kv=st.sampled_from([1, 2, 4, 8]),
+       g=st.sampled_from([1, 2, 3, 7, 8, 16]), grid=st.sampled_from([1, 7, 132, 148]))
+def test_schedule_properties_on_random_shapes(B, L, h_kv, g, grid):
+    """Any shape and CTA count: every item exactly once, no more lists than CTAs or items, each list
+    heaviest first where the items are packed or dealt round-robin, and plane groups in order where they
+    are dealt by group."""
+    h_q = g * h_kv
+    tiles = item_tiles(B, L, h_q, h_kv)
+    lists, grouped = G.prefill_schedule(B, L, h_q, h_kv, grid)
+    assert len(lists) == min(grid, len(tiles))
+    flat = np.concatenate([np.array(l, dtype=np.int64) for l in lists]) if lists else np.array([], np.int64)
+    assert np.array_equal(np.sort(flat), np.arange(len(tiles)))
+    planes = B * h_kv
+    for l in lists:
+        l = np.array(l, dtype=np.int64)
+        if grouped:
+            gp = group_planes(B, L, h_kv)
+            grp = (l % planes) // gp
+            assert np.all(np.diff(grp) >= 0)
+            for gg in np.unique(grp):
+                assert np.all(np.diff(tiles[l[grp == gg]]) <= 0)
+        elif len(l) > 1:
+            # packed lists are heaviest first; round-robin lists follow the item order, which is heaviest first too
+            assert np.all(np.diff(tiles[l]) <= 0)
